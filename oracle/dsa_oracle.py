@@ -1,0 +1,263 @@
+"""CPU oracle for the DeepSeek Sparse Attention (DSA) hot path.
+
+TEST INFRASTRUCTURE ONLY. This module is imported by the tests, by the smoke
+check and by the benchmark's CPU-baseline leg; the product path never calls it.
+It is a plain, slow, float64 statement of what the three stages compute. It
+shares no code with the CUDA library and imports nothing from it.
+
+Sources (the DeepSeek-V3.2-Exp pages; none prints an equation, so each stage is
+written from the words):
+  [jdon-indexer]   jdon.com "DeepSeek-V3.2-Exp", paragraph introducing the
+                   lightning indexer: light enough for FP8, very few heads, scores
+                   each query token against each earlier token with a weighted
+                   sum of ReLU-activated dot products.
+  [jdon-matchmake] same page, the "matchmaking" analogy paragraph: ReLU applied to
+                   the q_I/k_I meeting score, w_I as the weight, the highest scores
+                   go into the top-k set; main attention cost O(L^2) -> O(L*k).
+  [jdon-sparse]    same page, sparse-training paragraph: each query keeps only the
+                   2048 (K = 2048) highest-scoring earlier tokens.
+  [jdon-select]    same page, fine-grained selection paragraph: only the k chosen
+                   key/value entries take part; the output hidden state is u_t.
+  [jdon-causal]    same page, opening paragraph on cost: every token otherwise
+                   attends to all tokens before it (O(L^2)).
+  [openi-mla]      openi.cn "DeepSeek-V3.2", technical section, items on the
+                   lightning indexer (scores between the query token and earlier
+                   tokens), token selection (top-k value entries) and MLA in MQA
+                   mode (one value entry shared by many queries).
+  [mundobytes-run] mundobytes.com run guide: the serving command uses page size 64.
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * I[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]), ReLU per head before the
+    weighted sum; the FP8 per-token scales multiply the dequantised vectors.
+  * causal set s <= pos_t, inclusive of the query's own position.
+  * top-k order: score descending, then index ascending; -0 == +0; NaN lowest;
+    emitted in ascending index order, padded with -1 when pos_t + 1 < k.
+  * attention: key = full latent row (Dk dims), value = its first Dv dims, one
+    row shared by all heads; plain softmax with a caller-given scale, no sink.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ---------------------------------------------------------------------------
+# number formats
+
+
+def e4m3_value(byte: int) -> float:
+    """Value of one OCP FP8 E4M3 ("e4m3fn") byte, from the format definition:
+    1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 is
+    subnormal (m/8 * 2^-6); S.1111.111 is NaN; there is no infinity."""
+    s = (byte >> 7) & 1
+    e = (byte >> 3) & 0xF
+    m = byte & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        mag = (m / 8.0) * 2.0 ** (-6)
+    else:
+        mag = (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return -mag if s else mag
+
+
+E4M3_TABLE = np.array([e4m3_value(b) for b in range(256)], dtype=np.float64)
+
+
+def decode_e4m3(u8: np.ndarray) -> np.ndarray:
+    return E4M3_TABLE[np.asarray(u8, dtype=np.uint8)]
+
+
+def decode_bf16(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns -> float64 (bf16 is the top half of an IEEE binary32)."""
+    b = np.asarray(bits).view(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def dequant(u8_rows: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """x~ = s * dec(b) with one scale per leading row, in float64."""
+    x = decode_e4m3(u8_rows)
+    s = np.asarray(scale, dtype=np.float64).reshape((-1,) + (1,) * (x.ndim - 1))
+    return x * s
+
+
+# ---------------------------------------------------------------------------
+# stage 1: lightning indexer   [jdon-indexer], [jdon-matchmake], [openi-mla]
+
+
+def indexer_row(q_t: np.ndarray, w_t: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """Scores of one query token against `keys` (its causal prefix).
+
+    q_t  [H_I, d_I] float64: the token's indexer query heads (dequantised)
+    w_t  [H_I]      float64: the token's per-head weights
+    keys [n, d_I]   float64: indexer keys of positions 0..n-1 (dequantised)
+    returns I[s] = sum_j w_t[j] * max(0, q_t[j] . keys[s]),  s = 0..n-1
+    """
+    dots = keys @ q_t.T                      # [n, H_I]: q_I[t,j] . k_I[s]
+    return np.maximum(dots, 0.0) @ w_t       # ReLU per head, then the weighted sum
+
+
+# ---------------------------------------------------------------------------
+# stage 2: fine-grained token selection   [jdon-sparse], [jdon-select], [openi-mla]
+
+
+def topk_row(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices kept for one query row.
+
+    scores: float32 [n] — the row's scores over its causal prefix s = 0..n-1.
+    Returns int32 [k]: the m = min(k, n) indices that come first under the order
+    (score descending, index ascending), listed in ascending index order and
+    padded with -1. -0.0 and +0.0 compare equal; NaN ranks below every number.
+    """
+    v = np.asarray(scores, dtype=np.float32).astype(np.float64)
+    n = v.shape[0]
+    m = min(k, n)
+    idx = np.arange(n)
+    # primary key: -v ascending (NaN sorts last); secondary: index ascending
+    order = np.lexsort((idx, -v))
+    chosen = np.sort(order[:m])
+    out = np.full(k, -1, dtype=np.int32)
+    out[:m] = chosen
+    return out
+
+
+# ---------------------------------------------------------------------------
+# stage 3: sparse MQA attention over the latent rows   [jdon-select], [openi-mla]
+
+
+def sparse_attn_row(q_t: np.ndarray, kv_rows: np.ndarray, Dv: int, scale: float):
+    """Attention of one query token over its selected latent rows.
+
+    q_t     [H, Dk] float64: the token's query heads
+    kv_rows [m, Dk] float64: the selected rows (key = whole row, value = first Dv dims)
+    returns (o [H, Dv], lse [H]) with z = scale * q.k, o = softmax(z) @ v,
+    lse = log sum exp z (natural log). Two-pass softmax.
+    """
+    z = scale * (q_t @ kv_rows.T)                   # [H, m]
+    zmax = z.max(axis=1, keepdims=True)
+    p = np.exp(z - zmax)
+    Z = p.sum(axis=1, keepdims=True)
+    o = (p @ kv_rows[:, :Dv]) / Z
+    lse = zmax[:, 0] + np.log(Z[:, 0])
+    return o, lse
+
+
+def dense_causal_mqa_online(q_t: np.ndarray, kv_prefix: np.ndarray, Dv: int, scale: float):
+    """Dense causal MQA for one token, written as a one-key-at-a-time online
+    softmax (a different algorithm from `sparse_attn_row`). Used to pin the
+    invariant that DSA with k >= L equals dense causal attention."""
+    H = q_t.shape[0]
+    m = np.full(H, -np.inf)
+    l = np.zeros(H)
+    acc = np.zeros((H, Dv))
+    for s in range(kv_prefix.shape[0]):
+        z = scale * (q_t @ kv_prefix[s])
+        m_new = np.maximum(m, z)
+        a = np.exp(m - m_new)
+        b = np.exp(z - m_new)
+        l = l * a + b
+        acc = acc * a[:, None] + b[:, None] * kv_prefix[s, :Dv][None, :]
+        m = m_new
+    return acc / l[:, None], m + np.log(l)
+
+
+# ---------------------------------------------------------------------------
+# logical views of the key caches (contiguous or paged)  [mundobytes-run]
+
+
+def seq_keys(case: dict, b: int):
+    """Float64 indexer keys [len_b, d_I] and latent rows [len_b, Dk] of sequence b,
+    in logical position order. A paged cache maps position s to page
+    page_table[b, s // P], slot s % P; an indexer page holds P key rows of d_I
+    bytes followed by P little-endian float32 scales."""
+    L = int(case["seq_lens"][b])
+    fp8 = case["fp8"]
+    P = case["page_size"]
+    if P == 0:
+        if fp8:
+            kI = dequant(case["k_idx"][b, :L], case["k_scale"][b, :L])
+            kv = decode_bf16(case["kv"][b, :L])
+        else:
+            kI = np.asarray(case["k_idx"][b, :L], dtype=np.float64)
+            kv = np.asarray(case["kv"][b, :L], dtype=np.float64)
+        return kI, kv
+    d_I = case["d_I"]
+    pos = np.arange(L)
+    page = case["page_table"][b, pos // P].astype(np.int64)
+    slot = pos % P
+    pages = case["k_pages"]
+    kbytes = pages[page[:, None], slot[:, None] * d_I + np.arange(d_I)[None, :]]
+    sbytes = pages[page[:, None], P * d_I + slot[:, None] * 4 + np.arange(4)[None, :]]
+    scale = np.ascontiguousarray(sbytes).view("<f4").reshape(L)
+    kI = dequant(kbytes, scale)
+    kv = decode_bf16(case["kv"][page, slot])
+    return kI, kv
+
+
+def query_row(case: dict, t: int):
+    """Float64 (indexer query heads [H_I, d_I], weights [H_I], query heads [H, Dk]) of row t."""
+    if case["fp8"]:
+        qI = dequant(case["q_idx"][t][None], case["q_scale"][t:t + 1])[0]
+        q = decode_bf16(case["q"][t])
+    else:
+        qI = np.asarray(case["q_idx"][t], dtype=np.float64)
+        q = np.asarray(case["q"][t], dtype=np.float64)
+    w = np.asarray(case["w"][t], dtype=np.float64)
+    return qI, w, q
+
+
+# ---------------------------------------------------------------------------
+# whole path for chosen rows
+
+
+def forward_rows(case: dict, rows, keys_cache=None):
+    """Indexer -> top-k -> attention for query rows `rows` of `case`.
+
+    Returns {t: dict(scores=f64[pos+1], idx=int32[k], o=f64[H,Dv], lse=f64[H])}.
+    The selection runs on the oracle's own scores rounded to float32.
+    """
+    keys_cache = {} if keys_cache is None else keys_cache
+    out = {}
+    for t in rows:
+        b = int(case["row_seq"][t])
+        pos = int(case["pos"][t])
+        if b not in keys_cache:
+            keys_cache[b] = seq_keys(case, b)
+        kI, kv = keys_cache[b]
+        qI, w, q = query_row(case, t)
+        sc = indexer_row(qI, w, kI[:pos + 1])
+        idx = topk_row(sc.astype(np.float32), case["k"])
+        sel = idx[idx >= 0]
+        o, lse = sparse_attn_row(q, kv[sel], case["Dv"], case["softmax_scale"])
+        out[t] = dict(scores=sc, idx=idx, o=o, lse=lse)
+    return out
+
+
+def attn_rows_on_indices(case: dict, rows, idx_rows, keys_cache=None):
+    """Attention of `rows` recomputed on externally given index rows (e.g. a GPU's
+    selection): {t: (o [H,Dv], lse [H])}. Index -1 marks padding."""
+    keys_cache = {} if keys_cache is None else keys_cache
+    res = {}
+    for t, idx in zip(rows, idx_rows):
+        b = int(case["row_seq"][t])
+        if b not in keys_cache:
+            keys_cache[b] = seq_keys(case, b)
+        _, kv = keys_cache[b]
+        _, _, q = query_row(case, t)
+        idx = np.asarray(idx)
+        sel = idx[idx >= 0]
+        res[t] = sparse_attn_row(q, kv[sel], case["Dv"], case["softmax_scale"])
+    return res
+
+
+def indexer_rows(case: dict, rows, keys_cache=None):
+    """Indexer scores of `rows` over their causal prefixes: {t: f64[pos+1]}."""
+    keys_cache = {} if keys_cache is None else keys_cache
+    res = {}
+    for t in rows:
+        b = int(case["row_seq"][t])
+        pos = int(case["pos"][t])
+        if b not in keys_cache:
+            keys_cache[b] = seq_keys(case, b)
+        kI, _ = keys_cache[b]
+        qI, w, _ = query_row(case, t)
+        res[t] = indexer_row(qI, w, kI[:pos + 1])
+    return res

@@ -1,0 +1,345 @@
+"""Pins of the CPU oracle against things other than itself: published format
+tables, hand-worked cases, closed forms, library routines on special cases,
+brute-force enumeration and invariants the method's definition implies."""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _floats(tokens):
+    return [float(x) for x in tokens]
+
+
+# ----------------------------------------------------------------- formats
+
+def test_e4m3_against_ocp_table():
+    for line in open(os.path.join(GOLD, "e4m3_ocp_table.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        b, v = line.split()
+        got = O.e4m3_value(int(b, 16))
+        want = float(v)
+        if math.isnan(want):
+            assert math.isnan(got)
+        else:
+            assert got == want and math.copysign(1, got) == math.copysign(1, want), (b, got, want)
+
+
+def test_e4m3_table_against_torch_cast():
+    # torch's float8_e4m3fn -> float32 conversion is an independent implementation
+    allb = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = allb.view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+    mine = O.decode_e4m3(np.arange(256, dtype=np.uint8))
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(mine))
+    assert np.array_equal(ref[~nan], mine[~nan])
+    assert nan.sum() == 2  # 0x7F and 0xFF only
+
+
+def test_bf16_decode_against_torch():
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(4096, generator=g) * 100).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.decode_bf16(bits), x.to(torch.float64).numpy())
+
+
+def test_fp8_per_token_roundtrip_bound():
+    from sparse_long_context_04_b200.workloads import encode_e4m3_per_token
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((64, 128)).astype(np.float32)
+    q8, s = encode_e4m3_per_token(x)
+    xd = O.dequant(q8.numpy(), s.numpy())
+    # RNE to 3 mantissa bits: relative error <= 2^-4 for normals, absolute
+    # error <= 2^-10 * s in the subnormal range
+    err = np.abs(xd - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s.numpy()[:, None]) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    # the per-token maximum maps to 448 exactly
+    assert np.allclose(np.abs(xd).max(axis=1), np.abs(x).max(axis=1), rtol=1e-6)
+
+
+# ----------------------------------------------------------------- indexer
+
+def _hand_indexer():
+    d = {}
+    for line in open(os.path.join(GOLD, "indexer_hand_example.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, *vals = line.split()
+        d[key] = np.array(_floats(vals))
+    return d
+
+
+def test_indexer_hand_example_and_reading_guards():
+    d = _hand_indexer()
+    q = d["q"].reshape(2, 2)
+    k = d["k"].reshape(3, 2)
+    I = O.indexer_row(q, d["w"], k)
+    assert np.array_equal(I, d["I"])
+    assert not np.array_equal(I, d["relu_after_sum"])
+    assert not np.array_equal(I, d["no_relu"])
+
+
+def test_indexer_single_head_nonnegative_is_plain_matmul():
+    rng = np.random.default_rng(1)
+    q = np.abs(rng.standard_normal((1, 32)))
+    keys = np.abs(rng.standard_normal((50, 32)))
+    I = O.indexer_row(q, np.ones(1), keys)
+    ref = torch.from_numpy(keys) @ torch.from_numpy(q[0])   # library matmul
+    assert np.allclose(I, ref.numpy(), rtol=1e-13, atol=0)
+
+
+def test_indexer_relu_identities():
+    """relu(x) - relu(-x) = x and relu(x) + relu(-x) = |x| per head: negating one
+    head's query moves the score by w_j * (q_j . k); summing the score of q and -q
+    gives sum_j w_j |q_j . k|. A ReLU placed anywhere else breaks both."""
+    rng = np.random.default_rng(2)
+    H, d, n = 5, 16, 40
+    q = rng.standard_normal((H, d))
+    w = rng.standard_normal(H)
+    keys = rng.standard_normal((n, d))
+    base = O.indexer_row(q, w, keys)
+    for j in range(H):
+        qn = q.copy()
+        qn[j] = -qn[j]
+        diff = base - O.indexer_row(qn, w, keys)
+        assert np.allclose(diff, w[j] * np.einsum("sd,d->s", keys, q[j]), atol=1e-12)
+    both = base + O.indexer_row(-q, w, keys)
+    ref = np.abs(np.einsum("sd,hd->sh", keys, q)) @ w
+    assert np.allclose(both, ref, atol=1e-12)
+
+
+def test_indexer_linear_in_w_and_positively_homogeneous():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((4, 8))
+    keys = rng.standard_normal((30, 8))
+    w1, w2 = rng.standard_normal(4), rng.standard_normal(4)
+    assert np.allclose(O.indexer_row(q, w1 + w2, keys),
+                       O.indexer_row(q, w1, keys) + O.indexer_row(q, w2, keys), atol=1e-12)
+    assert np.allclose(O.indexer_row(2.5 * q, w1, keys), 2.5 * O.indexer_row(q, w1, keys), atol=1e-12)
+    assert np.allclose(O.indexer_row(q, w1, 0.25 * keys), 0.25 * O.indexer_row(q, w1, keys), atol=1e-12)
+
+
+def test_indexer_scale_folding():
+    """Per-token FP8 scales multiply the dequantised vectors: scores from (bytes,
+    scales) equal scores from pre-scaled vectors with unit scales."""
+    rng = np.random.default_rng(5)
+    qb = rng.integers(0, 256, size=(3, 4, 16)).astype(np.uint8)
+    kb = rng.integers(0, 256, size=(20, 16)).astype(np.uint8)
+    qb[(qb & 0x7F) == 0x7F] = 0  # no NaN bytes
+    kb[(kb & 0x7F) == 0x7F] = 0
+    sq = rng.uniform(0.01, 2, size=3).astype(np.float32)
+    sk = rng.uniform(0.01, 2, size=20).astype(np.float32)
+    w = rng.standard_normal(4)
+    keys = O.dequant(kb, sk)
+    for t in range(3):
+        q = O.dequant(qb[t][None], sq[t:t + 1])[0]
+        a = O.indexer_row(q, w, keys)
+        b = sq[t] * (np.maximum(O.decode_e4m3(kb) @ O.decode_e4m3(qb[t]).T * sk[:, None], 0) @ w)
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- top-k
+
+def _brute_topk(v, k):
+    """Enumerate every subset of size m = min(k, n); keep the unique one whose
+    members all precede all non-members under (score desc, index asc)."""
+    n = len(v)
+    m = min(k, n)
+
+    def before(a, b):  # does index a precede index b?
+        va, vb = v[a], v[b]
+        na, nb = math.isnan(va), math.isnan(vb)
+        if na != nb:
+            return nb          # a number precedes NaN
+        if not na and va != vb:
+            return va > vb
+        return a < b
+
+    winners = []
+    for sub in itertools.combinations(range(n), m):
+        rest = set(range(n)) - set(sub)
+        if all(before(a, b) for a in sub for b in rest):
+            winners.append(sub)
+    assert len(winners) == 1
+    out = list(winners[0]) + [-1] * (k - m)
+    return np.array(out, dtype=np.int32)
+
+
+def test_topk_hand_examples():
+    for line in open(os.path.join(GOLD, "topk_hand_examples.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, sc, exp = [p.strip() for p in line.split("|")]
+        v = np.array([float(x) for x in sc.split()], dtype=np.float32)
+        want = np.array([int(x) for x in exp.split()], dtype=np.int32)
+        assert np.array_equal(O.topk_row(v, int(k)), want), line
+
+
+def test_topk_brute_force_small_rows():
+    rng = np.random.default_rng(7)
+    pool = np.array([0.0, -0.0, 1.0, 1.0, -1.0, 2.5, np.inf, -np.inf, np.nan, 3.0, 1e-30],
+                    dtype=np.float32)
+    for trial in range(400):
+        n = int(rng.integers(1, 11))
+        if trial % 2:
+            v = rng.choice(pool, size=n)
+        else:
+            v = rng.integers(-2, 3, size=n).astype(np.float32)
+        k = int(rng.integers(1, 13))
+        assert np.array_equal(O.topk_row(v, k), _brute_topk([float(x) for x in v], k)), (v, k)
+
+
+def test_topk_short_rows_select_everything():
+    rng = np.random.default_rng(8)
+    for n in (1, 5, 63, 64):
+        v = rng.standard_normal(n).astype(np.float32)
+        out = O.topk_row(v, 64)
+        assert np.array_equal(out[:n], np.arange(n)) and np.all(out[n:] == -1)
+
+
+def test_topk_threshold_tie_across_k():
+    v = np.zeros(100, dtype=np.float32)
+    v[[3, 50, 97]] = 1.0
+    out = O.topk_row(v, 10)
+    assert np.array_equal(out, np.array([0, 1, 2, 3, 4, 5, 6, 7, 50, 97], dtype=np.int32))
+
+
+# ----------------------------------------------------------------- attention
+
+def test_attention_hand_example():
+    d = {}
+    for line in open(os.path.join(GOLD, "attention_hand_example.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, *vals = line.split()
+        d[key] = np.array(_floats(vals))
+    o, lse = O.sparse_attn_row(d["q"].reshape(1, 2), d["rows"].reshape(2, 2), 1, 1.0)
+    assert abs(o[0, 0] - d["o"][0]) < 1e-15 and abs(lse[0] - d["lse"][0]) < 1e-15
+
+
+def test_attention_against_torch_sdpa():
+    """Selected-row attention equals a library softmax-attention on the gathered
+    rows with key = whole row, value = first Dv dims."""
+    rng = np.random.default_rng(9)
+    H, Dk, Dv, m = 6, 24, 10, 37
+    q = rng.standard_normal((H, Dk))
+    rows = rng.standard_normal((m, Dk))
+    scale = 0.3
+    o, lse = O.sparse_attn_row(q, rows, Dv, scale)
+    qt = torch.from_numpy(q)[:, None, :]
+    kt = torch.from_numpy(rows)[None].expand(H, m, Dk)
+    vt = torch.from_numpy(rows[:, :Dv])[None].expand(H, m, Dv)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)[:, 0]
+    assert np.allclose(o, ref.numpy(), atol=1e-12)
+    ref_lse = torch.logsumexp(scale * (torch.from_numpy(q) @ torch.from_numpy(rows).T), dim=1)
+    assert np.allclose(lse, ref_lse.numpy(), atol=1e-12)
+
+
+def test_attention_single_row_and_two_row_closed_forms():
+    rng = np.random.default_rng(10)
+    q = rng.standard_normal((3, 8))
+    r = rng.standard_normal((2, 8))
+    o1, l1 = O.sparse_attn_row(q, r[:1], 5, 0.7)
+    assert np.array_equal(o1, np.broadcast_to(r[0, :5], (3, 5)))
+    assert np.allclose(l1, 0.7 * q @ r[0], atol=1e-14)
+    o2, l2 = O.sparse_attn_row(q, r, 5, 0.7)
+    z = 0.7 * q @ r.T
+    a = 1.0 / (1.0 + np.exp(z[:, 1] - z[:, 0]))
+    assert np.allclose(o2, a[:, None] * r[0, :5] + (1 - a)[:, None] * r[1, :5], atol=1e-14)
+    assert np.allclose(l2, np.log(np.exp(z[:, 0]) + np.exp(z[:, 1])), atol=1e-14)
+
+
+def test_attention_permutation_invariant():
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal((4, 16))
+    rows = rng.standard_normal((20, 16))
+    o, l = O.sparse_attn_row(q, rows, 8, 0.25)
+    p = rng.permutation(20)
+    o2, l2 = O.sparse_attn_row(q, rows[p], 8, 0.25)
+    assert np.allclose(o, o2, atol=1e-12) and np.allclose(l, l2, atol=1e-12)
+
+
+def test_dsa_with_k_at_least_L_is_dense_causal_mqa():
+    from sparse_long_context_04_b200.workloads import TINY, make_inputs
+    from tests.case_utils import case_from_inputs
+    spec = TINY.replace(lens=(40,), k=64)
+    case = case_from_inputs(make_inputs(spec))
+    res = O.forward_rows(case, range(40))
+    kI, kv = O.seq_keys(case, 0)
+    for t in (0, 1, 17, 39):
+        assert np.array_equal(res[t]["idx"][:t + 1], np.arange(t + 1))
+        _, _, q = O.query_row(case, t)
+        o, l = O.dense_causal_mqa_online(q, kv[:t + 1], spec.Dv, spec.softmax_scale)
+        assert np.allclose(res[t]["o"], o, atol=1e-12) and np.allclose(res[t]["lse"], l, atol=1e-12)
+
+
+# ----------------------------------------------------------------- causality, paging
+
+def test_causality_future_data_does_not_change_row():
+    from sparse_long_context_04_b200.workloads import TINY, make_inputs
+    from tests.case_utils import case_from_inputs
+    spec = TINY.replace(lens=(96,), k=16)
+    case = case_from_inputs(make_inputs(spec))
+    rows = [10, 50, 95]
+    a = O.forward_rows(case, rows)
+    rng = np.random.default_rng(12)
+    for t in rows[:2]:
+        case2 = dict(case)
+        case2["k_idx"] = case["k_idx"].copy()
+        case2["kv"] = case["kv"].copy()
+        case2["k_idx"][0, t + 1:] = rng.standard_normal(case2["k_idx"][0, t + 1:].shape)
+        case2["kv"][0, t + 1:] = rng.standard_normal(case2["kv"][0, t + 1:].shape)
+        b = O.forward_rows(case2, [t])[t]
+        for key in ("scores", "idx", "o", "lse"):
+            assert np.array_equal(a[t][key], b[key])
+
+
+def test_paged_and_contiguous_layouts_agree():
+    from sparse_long_context_04_b200.workloads import PAGED_DECODE_128K, make_inputs
+    from tests.case_utils import case_from_inputs
+    spec = PAGED_DECODE_128K.replace(batch=3, len_range=None, lens=(200, 64, 129), k=128,
+                                     plant_frac=0.05)
+    paged = case_from_inputs(make_inputs(spec))
+    contig = case_from_inputs(make_inputs(spec.replace(page_size=0)))
+    for b in range(3):
+        kp, vp = O.seq_keys(paged, b)
+        kc, vc = O.seq_keys(contig, b)
+        assert np.array_equal(kp, kc) and np.array_equal(vp, vc)
+    ra = O.forward_rows(paged, range(3))
+    rb = O.forward_rows(contig, range(3))
+    for t in range(3):
+        for key in ("scores", "idx", "o", "lse"):
+            assert np.array_equal(ra[t][key], rb[t][key])
+
+
+def test_paged_addressing_against_hand_built_pool():
+    """Build a tiny paged pool by hand (page size 4, a chosen page order) and
+    check the oracle's logical view recovers the rows in position order."""
+    P, d = 4, 16
+    L = 10
+    rng = np.random.default_rng(13)
+    kb = rng.integers(0, 0x70, size=(L, d)).astype(np.uint8)
+    sc = rng.uniform(0.5, 2, size=L).astype(np.float32)
+    kv = rng.integers(0, 2 ** 14, size=(L, 6)).astype(np.uint16)
+    order = [2, 0, 1]       # logical page i lives in physical page order[i]
+    pages = np.zeros((3, P * d + 4 * P), dtype=np.uint8)
+    kvpool = np.zeros((3, P, 6), dtype=np.uint16)
+    for s in range(L):
+        pg, sl = order[s // P], s % P
+        pages[pg, sl * d:(sl + 1) * d] = kb[s]
+        pages[pg, P * d + 4 * sl:P * d + 4 * sl + 4] = np.frombuffer(sc[s].tobytes(), np.uint8)
+        kvpool[pg, sl] = kv[s]
+    case = dict(fp8=True, page_size=P, d_I=d, seq_lens=np.array([L]), page_table=np.array([order]),
+                k_pages=pages, kv=kvpool)
+    kI, kvr = O.seq_keys(case, 0)
+    assert np.array_equal(kI, O.decode_e4m3(kb) * sc[:, None].astype(np.float64))
+    assert np.array_equal(kvr, O.decode_bf16(kv))
