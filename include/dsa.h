@@ -1,0 +1,177 @@
+/*
+ * dsa.h — C ABI of the DeepSeek Sparse Attention (DSA) hot path on B200 (sm_100a).
+ *
+ * The path has three stages, as the DeepSeek-V3.2-Exp pages describe them:
+ *   1. lightning indexer  I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]),  s <= pos_t
+ *        jdon.com "DeepSeek-V3.2-Exp", lightning-indexer paragraph (FP8, few heads,
+ *        weighted sum of ReLU-activated dot products) and the "matchmaking" analogy
+ *        paragraph (ReLU, w_I as weight, q_I and k_I scored on meeting);
+ *        openi.cn "DeepSeek-V3.2", technical section, lightning-indexer item.
+ *   2. fine-grained token selection: the k best-scoring earlier tokens per query
+ *        jdon.com, sparse-training paragraph (K = 2048) and selection paragraph;
+ *        openi.cn, token-selection item.
+ *   3. sparse MQA attention over the selected latent rows (all heads share one row)
+ *        jdon.com, selection paragraph (only the k chosen entries take part, output u_t);
+ *        openi.cn, "MLA in MQA mode" item (one value entry shared by many queries).
+ *
+ * Conventions (every entry point):
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller; the
+ *     library never allocates device memory and never frees caller memory.
+ *   - `stream` is a cudaStream_t passed as void*; all work is enqueued
+ *     asynchronously on it. NULL means the legacy default stream.
+ *   - Argument errors are found on the host before any launch and return
+ *     DSA_ERR_INVALID_ARG; valid shapes without a kernel return DSA_ERR_UNSUPPORTED.
+ *     Nothing is launched when an error is returned.
+ *   - Kernels check what only the device can see (sequence lengths against the
+ *     cache extent, page ids against the pool, indices against the causal range):
+ *     a violating access is skipped and recorded in a device error word, read
+ *     back with dsa_get_device_error(). Every on-device wait is bounded; a wait
+ *     that runs out records DSA_ERR_TIMEOUT there instead of hanging.
+ *   - No C++ exception crosses this boundary.
+ *
+ * Query rows and positions. A call covers T query rows. With cu_q == NULL
+ * (decode) row t is the newest token of sequence t: T == batch, pos_t =
+ * seq_lens[t] - 1. With cu_q != NULL (prefill) rows cu_q[b] .. cu_q[b+1]-1 belong
+ * to sequence b and are its last (cu_q[b+1]-cu_q[b]) tokens: the i-th of them sits
+ * at pos = seq_lens[b] - (cu_q[b+1]-cu_q[b]) + i. The causal set of a row is
+ * s = 0 .. pos_t, the row's own position included.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* bad pointer, size, stride or alignment */
+  DSA_ERR_UNSUPPORTED = 2,   /* valid arguments, no kernel for this shape/dtype */
+  DSA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, attribute) */
+  DSA_ERR_TIMEOUT = 4,       /* an on-device wait ran out (device error word) */
+  DSA_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required */
+  DSA_ERR_DEVICE_CHECK = 6   /* a device-side bounds check failed (device error word) */
+} dsa_status;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
+
+/* Addressing of the key caches, shared by all stages. */
+typedef struct {
+  int batch;              /* B >= 1 sequences */
+  const int *seq_lens;    /* device int32 [B]: keys held by each sequence (>= 1) */
+  const int *cu_q;        /* device int32 [B+1] query-row offsets (prefill); NULL = decode */
+  int page_size;          /* 0 = contiguous caches; 64 = paged caches */
+  const int *page_table;  /* device int32 [B][max_pages] physical page ids (paged only) */
+  int max_pages;          /* row length of page_table (paged only) */
+  int num_pages;          /* pages in each cache pool (paged only; ids must be < num_pages) */
+  int n_max;              /* host upper bound of seq_lens; contiguous caches are
+                             laid out [B][n_max][...] */
+} dsa_seq_layout;
+
+/*
+ * Stage 1 — lightning indexer scores.
+ *   scores[t*ld + s] = sum_j w[t*H_I + j] * max(0, q~[t,j,:] . k~[s,:])  for s <= pos_t,
+ * with q~ = q_scale[t] * dec(q_idx) and k~ = k_scale[s] * dec(k_idx) for E4M3
+ * (per-token fp32 scales, > 0), or the plain values for F32.
+ *   q_idx    device [T][H_I][d_I], E4M3 bytes or float32 (dt)
+ *   q_scale  device float32 [T] (E4M3) or NULL (F32)
+ *   k_idx    contiguous: device [B][n_max][d_I] (E4M3 bytes or float32);
+ *            paged (E4M3 only): pool of num_pages pages, each page_size*d_I key
+ *            bytes followed by page_size float32 scales (little-endian)
+ *   k_scale  contiguous E4M3: device float32 [B][n_max]; otherwise NULL
+ *   w        device float32 [T][H_I]
+ *   scores   device float32 [T][ld], ld >= n_max and a multiple of 4; entries with
+ *            s > pos_t are unspecified on return
+ * Fast path: E4M3 with H_I = 64, d_I = 128 (tcgen05 FP8 MMA). F32: H_I*d_I <= 8192,
+ * contiguous only. Buffers of the fast path must be 16-byte aligned.
+ */
+dsa_status dsa_indexer_scores(const void *q_idx, const float *q_scale,
+                              const void *k_idx, const float *k_scale, dsa_dtype dt,
+                              const float *w, int T, int H_I, int d_I,
+                              const dsa_seq_layout *lay, float *scores, long long ld,
+                              void *stream);
+
+/*
+ * Stage 2 — fine-grained top-k selection.
+ * For each row t reads scores[t*ld + s], s = 0..pos_t, and writes idx[t*k + i]:
+ * the m = min(k, pos_t+1) positions that come first under (score descending,
+ * position ascending), in ascending position order, then k-m entries of -1.
+ * -0.0 equals +0.0; NaN ranks below every number. Bit-exact, deterministic.
+ *   scores  device float32 [T][ld], 16-byte aligned, ld a multiple of 4
+ *   idx     device int32 [T][k]
+ * Rows up to 262144 keys; k >= 1.
+ */
+dsa_status dsa_topk(const float *scores, long long ld, int T, int k,
+                    const dsa_seq_layout *lay, int *idx, void *stream);
+
+/*
+ * Stage 3 — sparse MQA attention over the selected latent rows.
+ * For row t and head h, over the selected set S_t = {idx[t*k+i] >= 0}:
+ *   z_s = softmax_scale * (q[t,h,:] . kv[s,:])   (Dk dims),
+ *   out[t,h,:] = sum_s softmax(z)_s * kv[s, 0:Dv],  lse[t,h] = ln sum_s exp(z_s).
+ * A row whose S_t is empty gets out = 0 and lse = -inf.
+ *   q    device [T][H][Dk] (bf16 or float32: dt)
+ *   kv   contiguous: device [B][n_max][Dk]; paged (bf16 only): pool [num_pages][page_size][Dk]
+ *   idx  device int32 [T][k]: positions in the row's sequence, -1 = padding;
+ *        entries outside 0..pos_t are a device check failure
+ *   out  device [T][H][Dv], same dtype as q;  lse device float32 [T][H] or NULL
+ *   workspace  device scratch of at least dsa_sparse_mqa_attn_workspace_size() bytes
+ *              (256-byte aligned), or NULL when that size is 0
+ * Fast path: bf16, H = 128, Dk = 576, Dv = 512, 16-byte aligned rows (tcgen05 MMA).
+ * F32: H <= 1024, Dk <= 1024, Dv <= 1024, k <= 8192, contiguous only.
+ */
+size_t dsa_sparse_mqa_attn_workspace_size(int T, int H, int Dv, int k, dsa_dtype dt);
+dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt,
+                               int T, int H, int Dk, int Dv, float softmax_scale,
+                               const int *idx, int k, const dsa_seq_layout *lay,
+                               void *out, float *lse,
+                               void *workspace, size_t ws_bytes, void *stream);
+
+/* All three stages on one stream. */
+typedef struct {
+  /* indexer */
+  const void *q_idx; const float *q_scale;
+  const void *k_idx; const float *k_scale;
+  dsa_dtype idx_dt; const float *w; int H_I, d_I;
+  /* attention */
+  const void *q; const void *kv; dsa_dtype attn_dt;
+  int H, Dk, Dv; float softmax_scale;
+  /* selection and rows */
+  int k; int T;
+  dsa_seq_layout lay;
+  /* outputs */
+  void *out; float *lse;          /* lse may be NULL */
+  int *idx_out;                   /* optional device int32 [T][k] copy of the selection */
+} dsa_forward_args;
+
+/* Workspace bytes dsa_forward needs for these arguments (0 on invalid arguments). */
+size_t dsa_forward_workspace_size(const dsa_forward_args *a);
+
+/*
+ * Indexer -> top-k -> attention for a->T rows. Prefill rows are processed in
+ * chunks so that the score buffer stays within the workspace. The workspace is
+ * caller-owned device memory of at least dsa_forward_workspace_size(a) bytes,
+ * 256-byte aligned. No host synchronisation happens inside.
+ */
+dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_bytes,
+                       void *stream);
+
+/* Synchronises `stream`, then returns and clears the device error word:
+ * DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK (or DSA_ERR_CUDA if the
+ * synchronisation itself failed). */
+dsa_status dsa_get_device_error(void *stream);
+
+/* Upper bound, in nanoseconds, of every on-device wait (default 1e9). Applies to
+ * launches enqueued after the call. */
+dsa_status dsa_set_wait_limit_ns(unsigned long long ns);
+
+const char *dsa_status_string(dsa_status s);
+int dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H */

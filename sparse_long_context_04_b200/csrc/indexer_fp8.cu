@@ -1,0 +1,508 @@
+// Lightning indexer on the 5th-generation tensor cores (FP8 e4m3, tcgen05).
+//
+//   I[t,s] = s_q[t] * s_k[s] * sum_j w[t,j] * max(0, dec(q8[t,j,:]) . dec(k8[s,:]))
+//
+// jdon.com "DeepSeek-V3.2-Exp": the indexer is light enough to run in FP8 with
+// very few heads and scores each query token against each earlier token with a
+// weighted sum of ReLU-activated dot products (w_I the weight). The per-token
+// scales are positive, so ReLU(s_q s_k x) = s_q s_k ReLU(x) and they are applied
+// once per output.
+//
+// One MMA tile: D[128 keys, 64*G] = K8[128 keys, 128] . Q8[G tokens x 64 heads, 128]^T
+// (kind::f8f6f4, M = 128, N = 64G, K = 128 as four K = 32 steps), accumulated in
+// TMEM. The epilogue reads each key's row of D, applies ReLU, weights by w[t,:]
+// and sums the 64 heads of each token in registers, so the [t, j, s] tensor never
+// leaves the SM. G = 1 serves decode (one query per sequence); G = 4 serves
+// prefill (four consecutive query tokens of a sequence share each key tile).
+//
+// Work: the flat list of (query group, key tile) items of every sequence, key
+// tiles 0 .. floor(last position / 128) per group (causal), is split into one
+// contiguous range per persistent CTA. Item counts have a closed form, so each
+// CTA finds its range without a pre-pass.
+//
+// Roles: warp 0 issues TMA loads (keys: 64-row boxes, so a 128-key tile is two
+// loads, one per page in a paged cache; queries: one box per group), warp 1
+// allocates TMEM and issues the MMAs, the remaining warps run the epilogue.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kHI = 64;      // indexer heads
+constexpr int kDI = 128;     // indexer dim (bytes per e4m3 row)
+constexpr int kTileKeys = 128;
+
+template <int G>
+struct Cfg {
+  static constexpr int N = kHI * G;
+  static constexpr int kStages = G == 1 ? 8 : 4;
+  static constexpr int kEpiWarps = G == 1 ? 4 : 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kATile = kTileKeys * kDI;  // 16 KiB
+  static constexpr int kBTile = N * kDI;          // 8 or 32 KiB
+  static constexpr int kTmemCols = 2 * N;         // two accumulator buffers (128 or 512)
+  static constexpr int kData = kStages * kATile + 2 * kBTile;
+  static constexpr int kSmem = 1024 + kData + 1024;  // alignment slack + barriers
+  static constexpr uint32_t kIdesc = instr_desc(0, 0, 0, 0, 128, N);
+};
+
+struct Params {
+  const float *q_scale;   // [T]
+  const float *k_scale;   // contiguous [B][n_max]; nullptr when paged
+  const uint8_t *k_pool;  // paged pool base (scales live in the pages)
+  const float *w;         // [T][64]
+  float *scores;          // [T][ld]
+  long long ld;
+  int T;
+  Layout L;
+  ErrCtx e;
+};
+
+// ------------------------------------------------------------------ work walk
+// Rows of sequence b inside this launch, grouped G at a time from the first.
+struct SeqRows {
+  int Qc;              // query rows of the sequence in this launch (0 = none)
+  int r_lo;            // first local row
+  long long p_first;   // position of that row
+  int len;             // keys of the sequence
+};
+
+__device__ __forceinline__ SeqRows seq_rows(const Params &p, int b) {
+  SeqRows s;
+  const Layout &L = p.L;
+  s.len = __ldg(L.seq_lens + b);
+  s.Qc = 0;
+  s.r_lo = 0;
+  s.p_first = 0;
+  long long g_lo, g_hi, q0, Q;
+  if (L.cu_q == nullptr) {
+    q0 = b;
+    Q = 1;
+  } else {
+    q0 = __ldg(L.cu_q + b);
+    Q = __ldg(L.cu_q + b + 1) - q0;
+  }
+  g_lo = max(q0, (long long)L.row0);
+  g_hi = min(q0 + Q, (long long)L.row0 + p.T);
+  if (g_hi <= g_lo) return s;
+  if (s.len < 1 || s.len > cache_capacity(L) || Q > s.len) {
+    raise_error(p.e, DEV_BOUNDS, 0x400);
+    return s;
+  }
+  s.Qc = (int)(g_hi - g_lo);
+  s.r_lo = (int)(g_lo - L.row0);
+  s.p_first = s.len - Q + (g_lo - q0);
+  return s;
+}
+
+// F(n) = sum_{v=0}^{n-1} floor(v / P)
+__device__ __forceinline__ long long floor_prefix(long long n, long long P) {
+  const long long q = n / P, r = n % P;
+  return P * q * (q - 1) / 2 + q * r;
+}
+
+template <int G>
+struct GroupMath {
+  // key tiles of the first i groups of a sequence (all of them full groups)
+  __device__ static long long tiles_before(const SeqRows &s, long long i) {
+    const long long P = kTileKeys / G;
+    const long long u0 = (s.p_first + G - 1) / G;
+    return i + floor_prefix(u0 + i, P) - floor_prefix(u0, P);
+  }
+  __device__ static int groups(const SeqRows &s) { return (s.Qc + G - 1) / G; }
+  __device__ static long long last_pos(const SeqRows &s, int i) {
+    return min(s.p_first + (long long)(i + 1) * G - 1, s.p_first + s.Qc - 1);
+  }
+  __device__ static int tiles_of(const SeqRows &s, int i) { return (int)(last_pos(s, i) / kTileKeys) + 1; }
+  __device__ static long long tiles_total(const SeqRows &s) {
+    if (s.Qc == 0) return 0;
+    const int ng = groups(s);
+    return tiles_before(s, ng - 1) + tiles_of(s, ng - 1);
+  }
+};
+
+// A cursor over this CTA's items. All roles step identical cursors.
+template <int G>
+struct Cursor {
+  int b, i, kt, ntiles, ng;
+  SeqRows s;
+  long long left;  // items still to visit
+
+  __device__ void enter_seq(const Params &p, int nb) {
+    b = nb;
+    s = seq_rows(p, b);
+    ng = GroupMath<G>::groups(s);
+  }
+  // position at flat item f of sequence b (0 <= f < tiles_total)
+  __device__ void seek(const Params &p, int nb, long long f, long long count) {
+    enter_seq(p, nb);
+    int lo = 0, hi = ng - 1;  // largest i with tiles_before(i) <= f
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (GroupMath<G>::tiles_before(s, mid) <= f) lo = mid; else hi = mid - 1;
+    }
+    i = lo;
+    kt = (int)(f - GroupMath<G>::tiles_before(s, i));
+    ntiles = GroupMath<G>::tiles_of(s, i);
+    left = count;
+  }
+  // advance; returns true when the next item starts a new group
+  __device__ bool next(const Params &p) {
+    --left;
+    if (left <= 0) return false;
+    if (++kt < ntiles) return false;
+    kt = 0;
+    if (++i >= ng) {
+      i = 0;
+      do {
+        enter_seq(p, b + 1);
+      } while (ng == 0 && b + 1 < p.L.batch);
+    }
+    ntiles = GroupMath<G>::tiles_of(s, i);
+    return true;
+  }
+  __device__ int row0() const { return s.r_lo + i * G; }
+  __device__ int rows() const { return min(G, s.Qc - i * G); }
+};
+
+// ------------------------------------------------------------------ kernel
+template <int G>
+__global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
+    indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const Params p) {
+  using C = Cfg<G>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  unsigned char *sA = base;
+  unsigned char *sB = base + C::kStages * C::kATile;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + C::kData);
+  uint64_t *a_full = bars, *a_empty = bars + C::kStages;
+  uint64_t *b_full = bars + 2 * C::kStages, *b_empty = b_full + 2;
+  uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 2;
+  uint64_t *done_bar = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+  __shared__ long long s_range[2];  // first flat item of this CTA, number of items
+  __shared__ int s_seq;             // sequence holding the first item
+  __shared__ long long s_fseq;      // flat index of the first item within that sequence
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = p.L.batch;
+
+  // ---- work range: per-sequence item counts (closed form), block prefix sum
+  {
+    long long *pre = reinterpret_cast<long long *>(sA);  // aliases stage memory before any load
+    __shared__ long long part[32];
+    const int per = (B + blockDim.x - 1) / blockDim.x;
+    const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
+    long long acc = 0;
+    for (int b = b0; b < b1; ++b) {
+      const SeqRows s = seq_rows(p, b);
+      const long long n = GroupMath<G>::tiles_total(s);
+      pre[b] = n;
+      acc += n;
+    }
+    // exclusive scan of thread totals
+    long long incl = acc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) part[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x >> 5;
+      long long v = lane < nw ? part[lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long o = __shfl_up_sync(0xFFFFFFFFu, v, off);
+        if (lane >= off) v += o;
+      }
+      if (lane < nw) part[lane] = v;  // inclusive per-warp totals
+    }
+    __syncthreads();
+    long long run = (warp ? part[warp - 1] : 0) + incl - acc;
+    for (int b = b0; b < b1; ++b) {
+      const long long n = pre[b];
+      pre[b] = run;
+      run += n;
+    }
+    const long long W = part[(blockDim.x >> 5) - 1];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const long long f0 = W * blockIdx.x / gridDim.x;
+      const long long f1 = W * (blockIdx.x + 1) / gridDim.x;
+      int lo = 0, hi = B - 1;  // last sequence with pre[b] <= f0 (and items)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= f0) lo = mid; else hi = mid - 1;
+      }
+      while (lo + 1 < B && pre[lo + 1] <= f0) ++lo;
+      s_seq = lo;
+      s_fseq = f0 - pre[lo];
+      s_range[0] = f0;
+      s_range[1] = f1 - f0;
+    }
+    __syncthreads();
+  }
+  const long long n_items = s_range[1];
+
+  // ---- barriers and TMEM
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(a_full + s, 1);
+      mbar_init(a_empty + s, 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(b_full + j, 1);
+      mbar_init(b_empty + j, 1);
+      mbar_init(acc_full + j, 1);
+      mbar_init(acc_empty + j, C::kEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n_items > 0) {
+    if (warp == 0) {
+      // ================= producer (one lane)
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        Cursor<G> cur;
+        cur.seek(p, s_seq, s_fseq, n_items);
+        int gcount = 0;
+        bool new_group = true;
+        uint32_t a_last_par[C::kStages];
+        bool a_used[C::kStages];
+        for (int s = 0; s < C::kStages; ++s) a_used[s] = false;
+        bool ok = true;
+        for (long long n = 0; n < n_items && ok; ++n) {
+          if (new_group) {
+            const int slot = gcount & 1;
+            ok = mbar_wait(b_empty + slot, ((gcount >> 1) & 1) ^ 1, p.e, 0x410);
+            if (!ok) break;
+            mbar_expect_tx(b_full + slot, C::kBTile);
+            tma_load_2d(sB + slot * C::kBTile, &tm_q, b_full + slot, 0, cur.row0() * kHI);
+            ++gcount;
+          }
+          const int st = (int)(n % C::kStages);
+          const uint32_t use = (uint32_t)(n / C::kStages);
+          ok = mbar_wait(a_empty + st, (use & 1) ^ 1, p.e, 0x411);
+          if (!ok) break;
+          const int s0 = cur.kt * kTileKeys;
+          unsigned char *dst = sA + st * C::kATile;
+          int y0, y1 = -1;
+          if (p.L.page_size == 0) {
+            y0 = (int)((long long)cur.b * p.L.n_max + s0);
+            y1 = y0 + 64;
+          } else {
+            const int *pt = p.L.page_table + (long long)cur.b * p.L.max_pages;
+            const int pg0 = __ldg(pt + s0 / 64);
+            y0 = ((unsigned)pg0 < (unsigned)p.L.num_pages) ? pg0 * 66 : -1;
+            if (s0 + 64 < cur.s.len) {
+              const int pg1 = __ldg(pt + s0 / 64 + 1);
+              y1 = ((unsigned)pg1 < (unsigned)p.L.num_pages) ? pg1 * 66 : -2;
+            }
+            if (y0 == -1 || y1 == -2) raise_error(p.e, DEV_BOUNDS, 0x412);
+          }
+          const uint32_t bytes = (y0 >= 0 ? 8192u : 0u) + (y1 >= 0 ? 8192u : 0u);
+          mbar_expect_tx(a_full + st, bytes);
+          if (y0 >= 0) tma_load_2d(dst, &tm_k, a_full + st, 0, y0);
+          if (y1 >= 0) tma_load_2d(dst + 8192, &tm_k, a_full + st, 0, y1);
+          a_used[st] = true;
+          a_last_par[st] = use & 1;
+          new_group = cur.next(p);
+        }
+        // make sure no copy is still landing in shared memory before exit
+        for (int s = 0; s < C::kStages; ++s)
+          if (a_used[s]) mbar_wait(a_full + s, a_last_par[s], p.e, 0x413);
+        for (int j = 0; j < 2 && j < gcount; ++j) {
+          const int last = gcount - 1 - j;  // the last use of each B slot
+          mbar_wait(b_full + (last & 1), (last >> 1) & 1, p.e, 0x414);
+        }
+      }
+    } else if (warp == 1) {
+      // ================= MMA issuer (one lane)
+      if (lane == 0) {
+        Cursor<G> cur;
+        cur.seek(p, s_seq, s_fseq, n_items);
+        int gcount = 0;
+        bool new_group = true;
+        bool ok = true;
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        for (long long n = 0; n < n_items && ok; ++n) {
+          if (new_group) {
+            ok = mbar_wait(b_full + (gcount & 1), (gcount >> 1) & 1, p.e, 0x420);
+            if (!ok) break;
+            ++gcount;
+          }
+          const int slot = (gcount - 1) & 1;
+          const int st = (int)(n % C::kStages);
+          const uint32_t use = (uint32_t)(n / C::kStages);
+          const int ab = (int)(n & 1);
+          ok = mbar_wait(a_full + st, use & 1, p.e, 0x421);
+          if (!ok) break;
+          ok = mbar_wait(acc_empty + ab, (((uint32_t)(n >> 1)) & 1) ^ 1, p.e, 0x422);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(ab * C::N);
+#pragma unroll
+          for (int ks = 0; ks < kDI / 32; ++ks) {
+            const uint64_t ad = smem_desc(a0 + st * C::kATile + ks * 32, 16, 1024, SW_128B);
+            const uint64_t bd = smem_desc(b0 + slot * C::kBTile + ks * 32, 16, 1024, SW_128B);
+            umma_f8(d, ad, bd, C::kIdesc, ks > 0);
+          }
+          umma_commit(a_empty + st);
+          umma_commit(acc_full + ab);
+          new_group = cur.next(p);
+          if (new_group || n + 1 == n_items) umma_commit(b_empty + slot);
+        }
+        umma_commit(done_bar);
+        mbar_wait(done_bar, 0, p.e, 0x423);
+      }
+    } else {
+      // ================= epilogue warps
+      const int ew = warp - 2;
+      const int quad = warp & 3;         // TMEM lanes this warp may read
+      const int half = ew >> 2;          // G = 4: which pair of tokens
+      const int r = quad * 32 + lane;    // key row within the tile
+      constexpr int kTokPerWarp = G == 1 ? 1 : 2;
+      Cursor<G> cur;
+      cur.seek(p, s_seq, s_fseq, n_items);
+      for (long long n = 0; n < n_items; ++n) {
+        const int ab = (int)(n & 1);
+        if (!mbar_wait(acc_full + ab, ((uint32_t)(n >> 1)) & 1, p.e, 0x430)) break;
+        tc_fence_after();
+        const int s = cur.kt * kTileKeys + r;
+        const int b = cur.b;
+        // key scale
+        float sk = 0.f;
+        const bool key_ok = s < cur.s.len;
+        if (key_ok) {
+          if (p.L.page_size == 0) {
+            sk = __ldg(p.k_scale + (long long)b * p.L.n_max + s);
+          } else {
+            const int pg = __ldg(p.L.page_table + (long long)b * p.L.max_pages + s / 64);
+            if ((unsigned)pg < (unsigned)p.L.num_pages)
+              sk = __ldg(reinterpret_cast<const float *>(p.k_pool + (long long)pg * 8448 + 8192) + (s & 63));
+          }
+        }
+        const int nrows = cur.rows();
+#pragma unroll
+        for (int tt = 0; tt < kTokPerWarp; ++tt) {
+          const int g = G == 1 ? 0 : half * 2 + tt;
+          uint32_t v[2][32];
+          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + g * kHI);
+          tmem_ld32(taddr, v[0]);
+          tmem_ld32(taddr + 32, v[1]);
+          const int t = cur.row0() + g;
+          const float4 *w4 = reinterpret_cast<const float4 *>(p.w + (long long)min(t, p.T - 1) * kHI);
+          tmem_ld_wait();
+          float acc = 0.f;
+#pragma unroll
+          for (int j4 = 0; j4 < kHI / 4; ++j4) {
+            const float4 wv = __ldg(w4 + j4);
+            const uint32_t *vv = v[j4 >> 3] + (j4 & 7) * 4;
+            acc = fmaf(wv.x, fmaxf(__uint_as_float(vv[0]), 0.f), acc);
+            acc = fmaf(wv.y, fmaxf(__uint_as_float(vv[1]), 0.f), acc);
+            acc = fmaf(wv.z, fmaxf(__uint_as_float(vv[2]), 0.f), acc);
+            acc = fmaf(wv.w, fmaxf(__uint_as_float(vv[3]), 0.f), acc);
+          }
+          const long long pos = cur.s.p_first + (long long)cur.i * G + g;
+          if (g < nrows && key_ok && s <= pos)
+            p.scores[(long long)t * p.ld + s] = acc * __ldg(p.q_scale + t) * sk;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + ab);
+        cur.next(p);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows][128] with 128-byte swizzled boxes of box_rows rows.
+bool make_map(CUtensorMap *m, const void *ptr, unsigned long long rows, unsigned box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int G>
+cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int num_sms, cudaStream_t stream) {
+  using C = Cfg<G>;
+  CUtensorMap tq, tk;
+  const unsigned long long krows =
+      p.L.page_size ? (unsigned long long)p.L.num_pages * 66ull : (unsigned long long)p.L.batch * p.L.n_max;
+  if (!make_map(&tq, q, (unsigned long long)p.T * kHI, C::N)) return cudaErrorInvalidValue;
+  if (!make_map(&tk, kI, krows, 64)) return cudaErrorInvalidValue;
+  cudaError_t err =
+      cudaFuncSetAttribute(indexer_fp8_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (err != cudaSuccess) return err;
+  indexer_fp8_kernel<G><<<num_sms, C::kThreads, C::kSmem, stream>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int indexer_fp8_grid(int num_sms) { return num_sms; }
+
+cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uint8_t *kI, const float *k_scale,
+                               const float *w, int T, const Layout &L, float *scores, long long ld, const ErrCtx &e,
+                               int num_sms, cudaStream_t stream) {
+  if (L.batch > 8192) return cudaErrorInvalidValue;  // per-sequence prefix lives in stage memory
+  Params p;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.k_pool = kI;
+  p.w = w;
+  p.scores = scores;
+  p.ld = ld;
+  p.T = T;
+  p.L = L;
+  p.e = e;
+  if (L.cu_q == nullptr) return launch_g<1>(q, kI, p, num_sms, stream);
+  return launch_g<4>(q, kI, p, num_sms, stream);
+}
+
+}  // namespace dsa

@@ -1,0 +1,42 @@
+// Launchers behind the C ABI (host side). Each returns the CUDA error of its
+// launch; argument validation happens in dsa_api.cu before any of them runs.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace dsa {
+
+// top-k (topk.cu): C CTAs per row (cluster), `cap` keys of shared memory per CTA
+size_t topk_smem_bytes(int cap);
+cudaError_t launch_topk(const float *scores, long long ld, int T, int k, const Layout &L, int C, int cap, int *idx,
+                        const ErrCtx &e, cudaStream_t stream);
+
+// plain fp32 kernels on CUDA cores (fp32_path.cu)
+cudaError_t launch_indexer_f32(const float *q, const float *kI, const float *w, int T, int H_I, int d_I,
+                               const Layout &L, float *scores, long long ld, const ErrCtx &e, cudaStream_t stream);
+cudaError_t launch_attn_f32(const float *q, const float *kv, int T, int H, int Dk, int Dv, float scale,
+                            const int *idx, int k, const Layout &L, float *out, float *lse, const ErrCtx &e,
+                            cudaStream_t stream);
+
+// FP8 tcgen05 lightning indexer (indexer_fp8.cu): H_I = 64, d_I = 128
+int indexer_fp8_grid(int num_sms);
+cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uint8_t *kI, const float *k_scale,
+                               const float *w, int T, const Layout &L, float *scores, long long ld, const ErrCtx &e,
+                               int num_sms, cudaStream_t stream);
+
+// bf16 tcgen05 sparse MQA attention (attn_bf16.cu): H = 128, Dk = 576, Dv = 512
+struct AttnPlan {
+  int keys_per_split;  // multiple of 64, <= 256
+  int splits;          // per query row
+};
+AttnPlan attn_bf16_plan(int T, int k, int num_sms);
+size_t attn_bf16_workspace(int T, int k, int num_sms);
+cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, const int *idx, int k,
+                             const Layout &L, void *out, float *lse, void *ws, size_t ws_bytes, const ErrCtx &e,
+                             int num_sms, cudaStream_t stream);
+
+}  // namespace dsa
