@@ -30,8 +30,9 @@ __device__ __forceinline__ void raise_error(const ErrCtx &e, unsigned flag, unsi
   if (old == 0) atomicExch(e.word + 1, site);
 }
 
+// True once any wait has timed out: the remaining waits then give up at once.
 __device__ __forceinline__ bool error_raised(const ErrCtx &e) {
-  return *(volatile unsigned *)e.word != 0;
+  return (*(volatile unsigned *)e.word & DEV_TIMEOUT) != 0;
 }
 
 __device__ __forceinline__ unsigned long long globaltimer() {
