@@ -1,10 +1,428 @@
-// bf16 tcgen05 sparse MQA attention (placeholder until the kernel lands).
+// Sparse MQA attention over the selected latent rows on the tcgen05 tensor cores.
+//
+// jdon.com "DeepSeek-V3.2-Exp", selection paragraph: only the k chosen key/value
+// entries take part in attention; openi.cn "DeepSeek-V3.2", MLA-in-MQA-mode item:
+// one latent entry is shared by every query head. Each selected row is 576 bf16
+// values; the key is the whole row, the value its first 512 values.
+//
+// Work unit (one CTA): query row t and a split of up to 256 of its selected
+// positions. One pass, no running rescale:
+//   1. S[128 heads, n] = Q_t[128, 576] . K_sel[n, 576]^T  — nine 64-dim chunks,
+//      Q by TMA and the selected rows gathered with cp.async into 128-byte
+//      swizzled tiles; tcgen05 kind::f16, M = 128, N = n, accumulated in TMEM.
+//   2. Four warps (one head row per thread) read S from TMEM, take the row max
+//      and write P = exp(scale (S - max)) as bf16 into shared memory.
+//   3. O[128, 512] = P[128, n] . V[n, 512] with the value rows gathered again
+//      (MN-major B operand); O reuses the TMEM columns S occupied.
+//   4. O (unnormalised), the row max and the row sum go to the workspace; a
+//      second kernel merges the splits of each row with log-sum-exp weights.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
 #include "internal.h"
+
 namespace dsa {
-AttnPlan attn_bf16_plan(int, int, int) { return AttnPlan{256, 8}; }
-size_t attn_bf16_workspace(int, int, int) { return 0; }
-cudaError_t launch_attn_bf16(const void *, const void *, int, float, const int *, int, const Layout &, void *, float *,
-                             void *, size_t, const ErrCtx &, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kH = 128, kDk = 576, kDv = 512;
+constexpr int kRowBytes = kDk * 2;   // 1152
+constexpr int kMaxKeys = 256;        // keys per split
+constexpr int kChunks = kDk / 64;    // 9 dim chunks of 128 bytes
+constexpr int kStages = 3;
+constexpr int kQTile = kH * 128;               // 16 KiB
+constexpr int kKTile = kMaxKeys * 128;         // 32 KiB
+constexpr int kStage = kQTile + kKTile;        // 48 KiB
+constexpr int kRing = kStages * kStage;        // 144 KiB (also holds two 64 KiB value blocks)
+constexpr int kVBlock = 64 * kDv * 2;          // 64 KiB: 64 rows x 512 values
+constexpr int kPBytes = kH * kMaxKeys * 2;     // 64 KiB
+constexpr int kProducers = 128;                // warps 0-3
+constexpr int kMmaWarp = 4;
+constexpr int kThreads = 288;                  // + MMA warp + 4 softmax warps
+constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 8 + 256 + 1024;
+constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
+
+struct Params {
+  const __nv_bfloat16 *kv;
+  const int *idx;
+  int k;
+  int splits;
+  int keys_per_split;
+  float scale_log2;   // softmax_scale * log2(e)
+  float scale;
+  float *o_part;      // [rows][splits][128][512]
+  float2 *ml_part;    // [rows][splits][128]: (max * scale, sum)
+  Layout L;
+  ErrCtx e;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
 }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  unsigned char *ring = base;
+  unsigned char *sP = base + kRing;
+  long long *rows = reinterpret_cast<long long *>(sP + kPBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rows + kMaxKeys);
+  uint64_t *full = bars, *empty = bars + kStages;
+  uint64_t *vfull = bars + 2 * kStages, *vempty = vfull + 2;
+  uint64_t *s_full = vempty + 2, *p_full = s_full + 1, *o_full = p_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
+  __shared__ int s_nvalid;
+  __shared__ uint32_t s_valid[kMaxKeys / 32];  // bit i: selected entry i is a real row
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x / p.splits;     // row within this launch
+  const int split = blockIdx.x % p.splits;
+  const int k0 = split * p.keys_per_split;
+  const int nk = min(p.keys_per_split, p.k - k0);
+  const long long part = (long long)t * p.splits + split;
+
+  // ---- selected rows of this split (top-k output: valid positions first, then -1)
+  if (threadIdx.x == 0) s_nvalid = 0;
+  if (threadIdx.x < kMaxKeys / 32) s_valid[threadIdx.x] = 0;
+  __syncthreads();
+  const RowPos rp = row_position(p.L, t);
+  for (int i = threadIdx.x; i < kMaxKeys; i += kThreads) {
+    long long r = -1;
+    if (i < nk) {
+      const int s = __ldg(p.idx + (long long)t * p.k + k0 + i);
+      if (s >= 0 && s <= rp.pos && rp.len <= cache_capacity(p.L)) {
+        r = key_row(p.L, rp.b, s, p.e, 0x500);
+      } else if (s != -1) {
+        raise_error(p.e, DEV_BOUNDS, 0x501);
+      }
+    }
+    rows[i] = r;
+    if (r >= 0) {
+      atomicMax(&s_nvalid, i + 1);
+      atomicOr(&s_valid[i >> 5], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  const int nvalid = s_nvalid;  // entries at or after nvalid are all padding
+  if (nvalid == 0) {
+    if (threadIdx.x < kH) p.ml_part[part * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+    return;
+  }
+  const int nkb = (nvalid + 63) / 64;  // 64-key blocks
+  const int n = nkb * 64;              // MMA N of the score tile
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, kProducers + 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(vfull + j, kProducers);
+      mbar_init(vempty + j, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(o_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const char *kvb = reinterpret_cast<const char *>(p.kv);
+
+  if (warp < 4) {
+    // ================= producers: Q chunks by TMA, selected rows by cp.async
+    const int tid = threadIdx.x;
+    if (tid == 0) tma_prefetch_desc(&tm_q);
+    bool ok = true;
+    for (int c = 0; c < kChunks && ok; ++c) {
+      const int st = c % kStages;
+      ok = mbar_wait(empty + st, ((c / kStages) & 1) ^ 1, p.e, 0x510);
+      if (!ok) break;
+      unsigned char *sq = ring + st * kStage;
+      const uint32_t sk = smem_u32(sq + kQTile);
+      if (tid == 0) {
+        mbar_expect_tx(full + st, kQTile);
+        tma_load_2d(sq, &tm_q, full + st, c * 64, t * kH);
+      }
+      for (int q = tid; q < n * 8; q += kProducers) {
+        const int i = q >> 3, u = q & 7;
+        const long long r = rows[i];
+        const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + c * 128 + u * 16;
+        cp_async16_zfill(sk + sw128_off(i, u), src, r >= 0);
+      }
+      cp_async_arrive_noinc(full + st);
+    }
+    // value rows: wait until every score MMA has consumed the ring
+    if (ok) ok = mbar_wait(s_full, 0, p.e, 0x511);
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int st = kb & 1;
+      ok = mbar_wait(vempty + st, ((kb >> 1) & 1) ^ 1, p.e, 0x512);
+      if (!ok) break;
+      const uint32_t sv = smem_u32(ring + st * kVBlock);
+      for (int q = tid; q < 64 * 64; q += kProducers) {
+        const int i = q >> 6, u = q & 63;
+        const long long r = rows[kb * 64 + i];
+        const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + u * 16;
+        cp_async16_zfill(sv + (u >> 3) * 8192 + sw128_off(i, u & 7), src, r >= 0);
+      }
+      cp_async_arrive_noinc(vfull + st);
+    }
+    cp_async_wait_all();  // nothing may still land in shared memory after exit
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, 128, (uint32_t)n);
+      const uint32_t idesc_pv = instr_desc(1, 1, 0, 1, 128, 256);
+      const uint32_t r0 = smem_u32(ring), p0 = smem_u32(sP);
+      bool ok = true;
+      for (int c = 0; c < kChunks && ok; ++c) {
+        const int st = c % kStages;
+        ok = mbar_wait(full + st, (c / kStages) & 1, p.e, 0x520);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qa = r0 + st * kStage, ka = qa + kQTile;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_f16(tmem, smem_desc(qa + ks * 32, 16, 1024, SW_128B), smem_desc(ka + ks * 32, 16, 1024, SW_128B),
+                   idesc_qk, (c | ks) != 0);
+        umma_commit(empty + st);
+      }
+      umma_commit(s_full);
+      if (ok) ok = mbar_wait(p_full, 0, p.e, 0x521);
+      if (ok) tc_fence_after();
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int st = kb & 1;
+        ok = mbar_wait(vfull + st, (kb >> 1) & 1, p.e, 0x522);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t va = r0 + st * kVBlock, pa = p0 + kb * 16384;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = smem_desc(pa + ks * 32, 16, 1024, SW_128B);
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh)
+            umma_f16(tmem + nh * 256, ad, smem_desc(va + nh * 4 * 8192 + ks * 2048, 8192, 1024, SW_128B),
+                     idesc_pv, (kb | ks) != 0);
+        }
+        umma_commit(vempty + st);
+      }
+      umma_commit(o_full);
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax + output (warps 5..8, one head row per thread)
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    bool ok = mbar_wait(s_full, 0, p.e, 0x530);
+    if (ok) {
+      tc_fence_after();
+      for (int j = 0; j < n / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(trow + j * 32, v);
+        tmem_ld_wait();
+        const uint32_t vm = s_valid[j];
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if ((vm >> x) & 1u) m = fmaxf(m, __uint_as_float(v[x]));
+      }
+      const float mb = m * p.scale_log2;
+      for (int j = 0; j < n / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(trow + j * 32, v);
+        tmem_ld_wait();
+        const uint32_t vm = s_valid[j];
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float a = ((vm >> x) & 1u) ? exp2f(fmaf(__uint_as_float(v[x]), p.scale_log2, -mb)) : 0.f;
+          const float b = ((vm >> (x + 1)) & 1u) ? exp2f(fmaf(__uint_as_float(v[x + 1]), p.scale_log2, -mb)) : 0.f;
+          const uint32_t w = pack_bf16(a, b);
+          pk[x >> 1] = w;
+          __nv_bfloat162 bw = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+          l += __low2float(bw) + __high2float(bw);
+        }
+        // keys j*32 .. j*32+31 sit in 64-key block j/2, 16-byte chunks (j%2)*4 .. +3
+        unsigned char *pb = sP + (j >> 1) * 16384;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint32_t off = sw128_off((uint32_t)h, (uint32_t)((j & 1) * 4 + c4));
+          *reinterpret_cast<uint4 *>(pb + off) = make_uint4(pk[c4 * 4], pk[c4 * 4 + 1], pk[c4 * 4 + 2], pk[c4 * 4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      ok = mbar_wait(o_full, 0, p.e, 0x531);
+    }
+    if (ok) {
+      tc_fence_after();
+      float *orow = p.o_part + (part * kH + h) * kDv;
+      for (int j = 0; j < kDv / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(trow + j * 32, v);
+        tmem_ld_wait();
+        float4 *o4 = reinterpret_cast<float4 *>(orow + j * 32);
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          o4[x] = make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                              __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+      }
+      p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
+    } else {
+      p.ml_part[part * kH + h] = make_float2(-INFINITY, 0.f);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    // all MMAs have completed once o_full fired; if a wait gave up, wait here (bounded)
+    if (lane == 0) mbar_wait(o_full, 0, p.e, 0x540);
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge the splits of each (row, head): out = sum_c e^{m_c - M} O_c / sum_c e^{m_c - M} l_c.
+__global__ void __launch_bounds__(128)
+    attn_combine_kernel(const float *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
+                        __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  const int t = blockIdx.x, h = blockIdx.y;
+  __shared__ float wsh[64];
+  __shared__ float s_inv, s_lse;
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int c = 0; c < splits; ++c) M = fmaxf(M, ml_part[((long long)t * splits + c) * kH + h].x);
+    float Lsum = 0.f;
+    for (int c = 0; c < splits; ++c) {
+      const float2 ml = ml_part[((long long)t * splits + c) * kH + h];
+      const float wgt = (M == -INFINITY || ml.y == 0.f) ? 0.f : __expf(ml.x - M);
+      wsh[c] = wgt;
+      Lsum += wgt * ml.y;
+    }
+    s_inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    s_lse = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
+  }
+  __syncthreads();
+  const int d = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < splits; ++c) {
+    const float wgt = wsh[c];
+    if (wgt == 0.f) continue;
+    const float4 o = __ldcs(reinterpret_cast<const float4 *>(o_part + (((long long)t * splits + c) * kH + h) * kDv + d));
+    acc.x = fmaf(wgt, o.x, acc.x);
+    acc.y = fmaf(wgt, o.y, acc.y);
+    acc.z = fmaf(wgt, o.z, acc.z);
+    acc.w = fmaf(wgt, o.w, acc.w);
+  }
+  const float inv = s_inv;
+  __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(out + ((long long)t * kH + h) * kDv + d);
+  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  if (lse && threadIdx.x == 0) lse[(long long)t * kH + h] = s_lse;
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// q viewed as [rows][576] bf16, boxes of 64 values x 128 rows, 128-byte swizzle
+bool make_q_map(CUtensorMap *m, const void *q, unsigned long long rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDk, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+  cuuint32_t box[2] = {64, (cuuint32_t)kH};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t part_bytes_per_row(int splits) {
+  return (size_t)splits * kH * (kDv * sizeof(float) + sizeof(float2));
+}
+
+}  // namespace
+
+AttnPlan attn_bf16_plan(int T, int k, int num_sms) {
+  (void)T;
+  (void)num_sms;
+  AttnPlan pl;
+  pl.keys_per_split = k >= kMaxKeys ? kMaxKeys : ((k + 63) / 64) * 64;
+  pl.splits = (k + pl.keys_per_split - 1) / pl.keys_per_split;
+  return pl;
+}
+
+size_t attn_bf16_workspace(int T, int k, int num_sms) {
+  const AttnPlan pl = attn_bf16_plan(T, k, num_sms);
+  const int rows = T < kRowsPerLaunch ? T : kRowsPerLaunch;
+  return (size_t)rows * part_bytes_per_row(pl.splits);
+}
+
+cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, const int *idx, int k,
+                             const Layout &L, void *out, float *lse, void *ws, size_t ws_bytes, const ErrCtx &e,
+                             int num_sms, cudaStream_t stream) {
+  const AttnPlan pl = attn_bf16_plan(T, k, num_sms);
+  const int rows_max = T < kRowsPerLaunch ? T : kRowsPerLaunch;
+  if (ws_bytes < (size_t)rows_max * part_bytes_per_row(pl.splits)) return cudaErrorInvalidValue;
+  cudaError_t err = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (err != cudaSuccess) return err;
+  Params p;
+  p.kv = static_cast<const __nv_bfloat16 *>(kv);
+  p.k = k;
+  p.splits = pl.splits;
+  p.keys_per_split = pl.keys_per_split;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_part = static_cast<float *>(ws);
+  p.ml_part = reinterpret_cast<float2 *>(static_cast<char *>(ws) +
+                                         (size_t)rows_max * pl.splits * kH * kDv * sizeof(float));
+  p.e = e;
+  for (int r0 = 0; r0 < T; r0 += kRowsPerLaunch) {
+    const int nr = T - r0 < kRowsPerLaunch ? T - r0 : kRowsPerLaunch;
+    CUtensorMap tq;
+    const char *qc = static_cast<const char *>(q) + (size_t)r0 * kH * kRowBytes;
+    if (!make_q_map(&tq, qc, (unsigned long long)nr * kH)) return cudaErrorInvalidValue;
+    p.idx = idx + (size_t)r0 * k;
+    p.L = L;
+    p.L.row0 = L.row0 + r0;
+    attn_bf16_kernel<<<nr * pl.splits, kThreads, kSmem, stream>>>(tq, p);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    attn_combine_kernel<<<dim3(nr, kH), 128, 0, stream>>>(
+        p.o_part, p.ml_part, pl.splits, static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
+        lse ? lse + (size_t)r0 * kH : nullptr);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace dsa

@@ -136,7 +136,7 @@ dsa_status check_attn(const void *q, const void *kv, dsa_dtype dt, int H, int Dk
                       const Layout &L, const void *out) {
   if (!q || !kv || !idx || !out || H < 1 || Dk < 1 || Dv < 1 || Dv > Dk || k < 1) return DSA_ERR_INVALID_ARG;
   if (dt == DSA_BF16) {
-    if (H != 128 || Dk != 576 || Dv != 512) return DSA_ERR_UNSUPPORTED;
+    if (H != 128 || Dk != 576 || Dv != 512 || k > 16384) return DSA_ERR_UNSUPPORTED;
     if (!a16(q) || !a16(kv) || !a16(out)) return DSA_ERR_INVALID_ARG;
     return DSA_OK;
   }
