@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Throughput of the DSA hot path (lightning indexer -> top-k -> sparse MQA
+attention) on the 128K-context paged decode workload: B = 16 sequences of
+96K-128K keys, page size 64, k = 2048, 64 FP8 indexer heads of 128 dims,
+128 bf16 query heads over 576-wide latent rows.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of all three stages over the batch (each sequence's newest
+token). Prints one JSON line (rank 0). Under torchrun each rank processes its
+own batch (weak scaling, no data-path collective); the step time is the max over
+ranks. --impl reference times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "DSA tokens/s (indexer+top-k+sparse attn) at 128K decode, % of roofline"
+UNIT = "tokens/s"
+WORKLOAD = "paged_decode_b16_ctx96k_128k"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML (read-only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period=0.005):
+        super().__init__(daemon=True)
+        self.samples = []
+        self.period = period
+        self.stop_flag = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self.h = N.nvmlDeviceGetHandleByPciBusId(bus)
+            self.N = N
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def run(self):
+        if not self.ok:
+            return
+        N = self.N
+        while not self.stop_flag.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def summary(self, t0=None, t1=None):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        s = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not s:
+            s = self.samples
+        loaded = [x for x in s if not (x[2] & 0x1)] or s
+        mhz = statistics.median([x[1] for x in loaded]) if loaded else None
+        bits = 0
+        for x in loaded:
+            bits |= x[2]
+        reasons = [n for b, n in self.REASONS.items() if bits & b and b != 0x1]
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------ work accounting
+def algorithmic_bytes(inp):
+    """Bytes each stage must move (inputs read once, outputs written once)."""
+    s = inp.spec
+    lens = [int(x) for x in inp.seq_lens.tolist()]
+    B, tot = len(lens), sum(lens)
+    sel = sum(min(s.k, L) for L in lens)
+    pages = sum((L + s.page_size - 1) // s.page_size for L in lens) if s.page_size else 0
+    idx_bytes = (tot * (s.d_I + 4)            # FP8 key rows + per-key scale
+                 + B * (s.H_I * s.d_I + 4 + s.H_I * 4)   # query heads, scale, weights
+                 + pages * 4                  # page-table entries
+                 + tot * 4)                   # scores written
+    topk_bytes = tot * 4 + B * s.k * 4
+    attn_bytes = (sel * s.Dk * 2              # gathered latent rows
+                  + B * s.H * s.Dk * 2        # queries
+                  + B * s.k * 4 + pages * 4   # indices, page table
+                  + B * s.H * s.Dv * 2 + B * s.H * 4)  # output, lse
+    return {"indexer": idx_bytes, "topk": topk_bytes, "attn": attn_bytes}
+
+
+# ------------------------------------------------------------------ oracle (CPU) leg
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_rows(inp, budget_s, max_rows=None):
+    """Run the oracle's whole path on full query rows until `budget_s` is spent."""
+    from oracle import dsa_oracle as O
+    from tests.case_utils import case_from_inputs
+    case = case_from_inputs(inp)
+    rows = 0
+    t0 = time.perf_counter()
+    cache = {}
+    for t in range(inp.T):
+        O.forward_rows(case, [t], cache)
+        cache.clear()
+        rows += 1
+        if time.perf_counter() - t0 > budget_s or (max_rows and rows >= max_rows):
+            break
+    return rows, time.perf_counter() - t0
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--len-range", type=int, nargs=2, default=None,
+                    help="override the context-length range (profiling on a smaller case)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import datetime
+
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    from sparse_long_context_04_b200 import build as B
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    from sparse_long_context_04_b200 import device as G
+    from sparse_long_context_04_b200 import dsa as D
+    from sparse_long_context_04_b200 import workloads as W
+
+    spec = W.WORKLOADS[WORKLOAD]
+    spec = spec.replace(seed=spec.seed + 1000 * rank)
+    if args.len_range:
+        spec = spec.replace(len_range=tuple(args.len_range))
+    inp = W.make_inputs(spec)
+    dc = G.to_device(inp, dev)
+    T, s = dc.T, spec
+    scores = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, s.k), dtype=torch.int32, device=dev)
+    out = torch.empty((T, s.H, s.Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
+    wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
+    ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, scores)
+        if ev is not None:
+            ev[1].record(stream)
+        D.dsa_topk(scores, s.k, dc.layout, idx)
+        if ev is not None:
+            ev[2].record(stream)
+        D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if D.dsa_get_device_error() != D.DSA_OK:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wt0 = time.perf_counter()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    wt1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if D.dsa_get_device_error() != D.DSA_OK:
+        raise RuntimeError("device error during timing")
+
+    # ---- end to end through dsa_forward with host buffers
+    fw = G.Forward(dc, keep_idx=False)
+    host_in = {n: getattr(dc, n).cpu().pin_memory() for n in ("q_idx", "q_scale", "w", "q")}
+    host_in["seq_lens"] = dc.layout.seq_lens.cpu().pin_memory()
+    host_in["page_table"] = dc.layout.page_table.cpu().pin_memory()
+    dev_in = {"q_idx": dc.q_idx, "q_scale": dc.q_scale, "w": dc.w, "q": dc.q,
+              "seq_lens": dc.layout.seq_lens, "page_table": dc.layout.page_table}
+    out_h = torch.empty(fw.out.shape, dtype=fw.out.dtype).pin_memory()
+    lse_h = torch.empty(fw.lse.shape, dtype=fw.lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def e2e_step():
+        for n, h in host_in.items():
+            dev_in[n].copy_(h, non_blocking=True)
+        fw(stream)
+        out_h.copy_(fw.out, non_blocking=True)
+        lse_h.copy_(fw.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    sampler.stop_flag.set()
+    sampler.join()
+    if D.dsa_get_device_error() != D.DSA_OK:
+        raise RuntimeError("device error during the end-to-end loop")
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    hbm, hbm_src = peaks()
+    ab = algorithmic_bytes(inp)
+    step_s = ms / 1e3 / args.steps
+    idx_s = stage_ms[0] / 1e3
+    idx_gbs = ab["indexer"] / idx_s / 1e9
+    ta_s = (stage_ms[1] + stage_ms[2]) / 1e3
+    ta_gbs = (ab["topk"] + ab["attn"]) / ta_s / 1e9
+    step_gbs = sum(ab.values()) / step_s / 1e9
+    res = {
+        "metric": METRIC,
+        "value": world * T * args.steps / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 indexer + bf16 attention (fp32 accumulate)",
+        "data": "synthetic (seeded; shapes and planted structure of the 128K paged decode workload)",
+        "config": {
+            "workload": WORKLOAD if not args.len_range else WORKLOAD + "@len%d-%d" % tuple(args.len_range),
+            "batch_per_gpu": T, "context": "uniform %d..%d" % spec.len_range,
+            "keys_total_per_gpu": int(inp.seq_lens.sum()), "page_size": s.page_size, "k": s.k,
+            "H_I": s.H_I, "d_I": s.d_I, "H": s.H, "Dk": s.Dk, "Dv": s.Dv,
+            "parallelism": f"dp{world} (independent sequences per rank)",
+            "l2": "inputs larger than L2: the 242 MB paged indexer-key cache is streamed every step",
+        },
+        "stages_us": {"indexer": stage_ms[0] * 1e3, "topk": stage_ms[1] * 1e3, "attention": stage_ms[2] * 1e3},
+        "roofline": {
+            "bound": "hbm", "kernel": "indexer_fp8_kernel (decode, N=64)",
+            "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
+            "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured" else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": ab["indexer"],
+            "traffic": None,
+        },
+        "topk_attn_roofline": {"achieved": ta_gbs, "frac": ta_gbs / hbm,
+                               "algorithmic_bytes": ab["topk"] + ab["attn"]},
+        "step_roofline": {"achieved": step_gbs, "frac": step_gbs / hbm, "algorithmic_bytes": sum(ab.values())},
+        "e2e": {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                "api": "dsa_forward"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": sampler.summary(wt0, wt1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rows, secs = oracle_rows(inp, args.cpu_budget)
+        res["cpu_baseline"] = {
+            "value": rows / secs, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {T} query rows of this workload, whole path per row (fp64 numpy), {secs:.1f} s"}
+    print(json.dumps(res), flush=True)
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as it stands, on a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    from oracle import dsa_oracle as O
+    from sparse_long_context_04_b200 import workloads as W
+    from tests.case_utils import case_from_inputs
+
+    spec = W.WORKLOADS[WORKLOAD]
+    inp = W.make_inputs(spec)
+    case = case_from_inputs(inp)
+    # one step = the oracle's whole path on a slice of one query row's keys,
+    # sized so that warm-up plus timed steps take about two minutes
+    t_probe = time.perf_counter()
+    O.forward_rows(case, [0])
+    row_s = time.perf_counter() - t_probe
+    n_steps = args.steps + args.warmup
+    frac = min(1.0, 120.0 / max(1e-9, n_steps * row_s))
+    lens = [int(x) for x in inp.seq_lens.tolist()]
+
+    def sample_step(i):
+        t = i % inp.T
+        b = int(case["row_seq"][t])
+        kI, kv = O.seq_keys(case, b)
+        m = max(1, int(lens[b] * frac))
+        qI, w, q = O.query_row(case, t)
+        sc = O.indexer_row(qI, w, kI[:m])
+        ix = O.topk_row(sc.astype("float32"), spec.k)
+        sel = ix[ix >= 0]
+        O.sparse_attn_row(q, kv[sel], spec.Dv, spec.softmax_scale)
+        return m
+
+    for i in range(args.warmup):
+        sample_step(i)
+    keys = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        keys += sample_step(i)
+    secs = time.perf_counter() - t0
+    mean_len = sum(lens) / len(lens)
+    value = keys / mean_len / secs    # query rows per second at the workload's mean context
+    cores = _blas_threads()
+    res = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes and planted structure of the 128K paged decode workload)",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": inp.T, "k": spec.k, "page_size": spec.page_size},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: one query row, indexer over the first {frac:.3f} of its keys, "
+                                   f"top-k and attention; scaled to rows/s at the mean context {mean_len:.0f}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
