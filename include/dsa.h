@@ -53,7 +53,8 @@ typedef enum {
   DSA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, attribute) */
   DSA_ERR_TIMEOUT = 4,       /* an on-device wait ran out (device error word) */
   DSA_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required */
-  DSA_ERR_DEVICE_CHECK = 6   /* a device-side bounds check failed (device error word) */
+  DSA_ERR_DEVICE_CHECK = 6,  /* a device-side bounds check failed (device error word) */
+  DSA_ERR_TOO_LARGE = 7      /* the call needs more scratch than the library's built-in array */
 } dsa_status;
 
 typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
@@ -129,6 +130,33 @@ dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt,
                                const int *idx, int k, const dsa_seq_layout *lay,
                                void *out, float *lse,
                                void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Stage 3 without a caller workspace (no counterpart on the pages; this entry
+ * point exists for callers, not for the method).
+ * Same computation, arguments and dtype as dsa_sparse_mqa_attn with dt = DSA_BF16,
+ * minus the workspace: the per-split partial results go to a scratch array of
+ * DSA_NOALLOC_SCRATCH_BYTES (40 MiB) that the library owns as a static device
+ * variable, so this call never allocates device memory. It is for callers that
+ * may not allocate: code running under a host framework that has reserved all
+ * device memory up front, or a serving loop where cudaMalloc's implicit device
+ * synchronisation is not allowed. Every GPU that loads the library holds the
+ * 40 MiB until the process exits.
+ *   - A call needs T * ceil(k/256) * 263168 bytes of scratch (16 decode rows at
+ *     k = 2048 fit); larger calls return DSA_ERR_TOO_LARGE and launch nothing.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array: calls whose kernels may overlap on the GPU
+ *     (other streams, other host threads) race on it and must be serialised by
+ *     the caller. Nothing in it needs to start at zero.
+ * Only DSA_BF16 with H = 128, Dk = 576, Dv = 512 is accepted.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (40ull << 20)
+dsa_status dsa_sparse_mqa_attn_noalloc(const void *q, const void *kv, dsa_dtype dt,
+                                       int T, int H, int Dk, int Dv, float softmax_scale,
+                                       const int *idx, int k, const dsa_seq_layout *lay,
+                                       void *out, float *lse, void *stream);
 
 /* All three stages on one stream. */
 typedef struct {

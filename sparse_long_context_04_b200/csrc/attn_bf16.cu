@@ -18,6 +18,7 @@
 //      second kernel merges the splits of each row with log-sum-exp weights.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <mutex>
 #include <math.h>
 
 #include "common.cuh"
@@ -423,6 +424,81 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
+}
+
+
+// ------------------------------------------------------------------ built-in scratch
+// For callers that may not allocate device memory: the split partials live in
+// this file-scope array instead of a caller workspace. Host code must not pass
+// the symbol itself to a kernel (on the host it names a shadow variable, not
+// device memory): its device address is looked up once per device below.
+namespace {
+constexpr size_t kScratchBytes = size_t(40) << 20;  // 40 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
+
+constexpr int kScratchDevices = 64;
+void *g_scratch_addr[kScratchDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device, with that device current).
+cudaError_t scratch_address(void **out) {
+  int dev = -1;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void *ptr = nullptr;
+    err = cudaGetSymbolAddress(&ptr, g_attn_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t attn_bf16_scratch_limit() { return kScratchBytes; }
+
+size_t attn_bf16_scratch_bytes(int T, int k) {
+  const AttnPlan pl = attn_bf16_plan(T, k, 0);
+  return (size_t)T * part_bytes_per_row(pl.splits);
+}
+
+cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float scale, const int *idx, int k,
+                                     const Layout &L, void *out, float *lse, const ErrCtx &e, int num_sms,
+                                     cudaStream_t stream) {
+  (void)num_sms;
+  const AttnPlan pl = attn_bf16_plan(T, k, num_sms);
+  const size_t need = (size_t)T * part_bytes_per_row(pl.splits);
+  if (need > kScratchBytes) return cudaErrorInvalidValue;
+  void *scratch = nullptr;
+  cudaError_t err = scratch_address(&scratch);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (err != cudaSuccess) return err;
+  CUtensorMap tq;
+  if (!make_q_map(&tq, q, (unsigned long long)T * kH)) return cudaErrorInvalidValue;
+  Params p;
+  p.kv = static_cast<const __nv_bfloat16 *>(kv);
+  p.idx = idx;
+  p.k = k;
+  p.splits = pl.splits;
+  p.keys_per_split = pl.keys_per_split;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_part = static_cast<float *>(scratch);
+  p.ml_part = reinterpret_cast<float2 *>(static_cast<char *>(scratch) +
+                                         (size_t)T * pl.splits * kH * kDv * sizeof(float));
+  p.L = L;
+  p.e = e;
+  attn_bf16_kernel<<<T * pl.splits, kThreads, kSmem, stream>>>(tq, p);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  attn_combine_kernel<<<dim3(T, kH), 128, 0, stream>>>(p.o_part, p.ml_part, pl.splits,
+                                                        static_cast<__nv_bfloat16 *>(out), lse);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa

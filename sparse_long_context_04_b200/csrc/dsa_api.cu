@@ -214,6 +214,7 @@ const char *dsa_status_string(dsa_status s) {
     case DSA_ERR_TIMEOUT: return "on-device wait timed out";
     case DSA_ERR_WORKSPACE: return "workspace missing or too small";
     case DSA_ERR_DEVICE_CHECK: return "device-side bounds check failed";
+    case DSA_ERR_TOO_LARGE: return "call needs more scratch than the built-in scratch array holds";
   }
   return "unknown status";
 }
@@ -287,6 +288,24 @@ dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt, int 
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
   return run_attn(q, kv, dt, T, H, Dk, Dv, softmax_scale, idx, k, L, out, lse, workspace, ws_bytes, e, sms,
                   static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_mqa_attn_noalloc(const void *q, const void *kv, dsa_dtype dt, int T, int H, int Dk, int Dv,
+                                       float softmax_scale, const int *idx, int k, const dsa_seq_layout *lay,
+                                       void *out, float *lse, void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  s = check_attn(q, kv, dt, H, Dk, Dv, idx, k, L, out);
+  if (s != DSA_OK) return s;
+  if (dt != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  if (dsa::attn_bf16_scratch_bytes(T, k) > dsa::attn_bf16_scratch_limit()) return DSA_ERR_TOO_LARGE;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_attn_bf16_noalloc(q, kv, T, softmax_scale, idx, k, L, out, lse, e, sms,
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 size_t dsa_forward_workspace_size(const dsa_forward_args *a) {

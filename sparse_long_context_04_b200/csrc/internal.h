@@ -39,4 +39,11 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
                              const Layout &L, void *out, float *lse, void *ws, size_t ws_bytes, const ErrCtx &e,
                              int num_sms, cudaStream_t stream);
 
+// same attention with its partials in the library's static scratch array
+size_t attn_bf16_scratch_bytes(int T, int k);
+size_t attn_bf16_scratch_limit();
+cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float scale, const int *idx, int k,
+                                     const Layout &L, void *out, float *lse, const ErrCtx &e, int num_sms,
+                                     cudaStream_t stream);
+
 }  // namespace dsa

@@ -16,7 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_WORKSPACE, \
-    DSA_ERR_DEVICE_CHECK = range(7)
+    DSA_ERR_DEVICE_CHECK, DSA_ERR_TOO_LARGE = range(8)
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
 
 
@@ -56,7 +56,7 @@ _lib = None
 
 EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size", "dsa_sparse_mqa_attn",
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
-           "dsa_status_string", "dsa_version")
+           "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc")
 
 
 def lib() -> ctypes.CDLL:
@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_mqa_attn_workspace_size.restype = sz
         L.dsa_sparse_mqa_attn.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i, ctypes.POINTER(SeqLayout),
                                           vp, vp, vp, sz, vp]
+        L.dsa_sparse_mqa_attn_noalloc.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i,
+                                                  ctypes.POINTER(SeqLayout), vp, vp, vp]
+        L.dsa_sparse_mqa_attn_noalloc.restype = i
         L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(ForwardArgs)]
         L.dsa_forward_workspace_size.restype = sz
         L.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
@@ -162,6 +165,16 @@ def dsa_sparse_mqa_attn(q, kv, idx, layout: Layout, out, lse, softmax_scale, wor
                                   ctypes.byref(layout.c), _p(out), _p(lse), _p(workspace), ws_bytes,
                                   _stream(stream))
     _check(s, "dsa_sparse_mqa_attn")
+
+
+def dsa_sparse_mqa_attn_noalloc(q, kv, idx, layout: Layout, out, lse, softmax_scale, stream=None):
+    """Stage 3 with the library's built-in scratch instead of a caller workspace
+    (for callers that may not allocate device memory; see include/dsa.h)."""
+    T, H, Dk = (int(x) for x in q.shape)
+    s = lib().dsa_sparse_mqa_attn_noalloc(_p(q), _p(kv), _dt(q), T, H, Dk, int(out.shape[2]),
+                                          float(softmax_scale), _p(idx), int(idx.shape[1]),
+                                          ctypes.byref(layout.c), _p(out), _p(lse), _stream(stream))
+    _check(s, "dsa_sparse_mqa_attn_noalloc")
 
 
 def forward_args(q_idx, q_scale, k_idx, k_scale, w, q, kv, k, softmax_scale, layout: Layout, out, lse=None,
