@@ -192,6 +192,11 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_byt
  * synchronisation itself failed). */
 dsa_status dsa_get_device_error(void *stream);
 
+/* As dsa_get_device_error, and also writes (when site != NULL) the code of the
+ * first device check or wait that failed (0 when none): a diagnostic for bug
+ * reports. */
+dsa_status dsa_get_device_error_site(void *stream, unsigned *site);
+
 /* Upper bound, in nanoseconds, of every on-device wait (default 1e9). Applies to
  * launches enqueued after the call. */
 dsa_status dsa_set_wait_limit_ns(unsigned long long ns);

@@ -71,23 +71,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As above, but the thread may sleep up to `hint_ns` waiting for the phase,
+// instead of polling: waiting warps then leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
-// Waits for the phase with the given parity to complete. Returns false (after
-// recording DEV_TIMEOUT with `site`) when the wait exceeds the limit, or at once
-// when another wait has already failed, so that every role can wind down.
-static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const ErrCtx &e, unsigned site) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: sleeping waits, each at most 1 ms, until the phase
+// completes, another wait has timed out, or the deadline passes (DEV_TIMEOUT
+// recorded with `site`).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const ErrCtx &e, unsigned site) {
   const unsigned long long t0 = globaltimer();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (error_raised(e)) return false;
     if (globaltimer() - t0 > e.limit) {
       raise_error(e, DEV_TIMEOUT, site);
       return false;
     }
   }
+}
+
+// Waits for the phase with the given parity to complete. Returns false (after
+// recording DEV_TIMEOUT with `site`) when the wait exceeds the limit, or at once
+// when another wait has already timed out, so that every role can wind down.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const ErrCtx &e, unsigned site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, e, site);
+}
+
+// Waits (bounded) until the shared counter *c equals `target` (a turn counter
+// that orders work handed out to several warps).
+__device__ __forceinline__ bool wait_turn(const volatile int *c, int target, const ErrCtx &e, unsigned site) {
+  if (*c == target) return true;
+  const unsigned long long t0 = globaltimer();
+  while (*c != target) {
+    __nanosleep(64);
+    if (error_raised(e)) return false;
+    if (globaltimer() - t0 > e.limit) {
+      raise_error(e, DEV_TIMEOUT, site);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------- proxies / fences
@@ -185,6 +219,15 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+// Plain (untiled) bulk copy global -> shared, completing on `bar` with tx bytes.
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {

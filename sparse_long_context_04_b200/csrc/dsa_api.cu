@@ -225,7 +225,8 @@ dsa_status dsa_set_wait_limit_ns(unsigned long long ns) {
   return DSA_OK;
 }
 
-dsa_status dsa_get_device_error(void *stream) {
+dsa_status dsa_get_device_error_site(void *stream, unsigned *site) {
+  if (site) *site = 0;
   ErrCtx e;
   int sms;
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
@@ -234,10 +235,13 @@ dsa_status dsa_get_device_error(void *stream) {
   unsigned h[2] = {0, 0};
   if (cudaMemcpy(h, e.word, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
   if (h[0] == 0) return DSA_OK;
+  if (site) *site = h[1];
   const unsigned zero[2] = {0, 0};
   if (cudaMemcpy(e.word, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
   return (h[0] & dsa::DEV_TIMEOUT) ? DSA_ERR_TIMEOUT : DSA_ERR_DEVICE_CHECK;
 }
+
+dsa_status dsa_get_device_error(void *stream) { return dsa_get_device_error_site(stream, nullptr); }
 
 dsa_status dsa_indexer_scores(const void *q_idx, const float *q_scale, const void *k_idx, const float *k_scale,
                               dsa_dtype dt, const float *w, int T, int H_I, int d_I, const dsa_seq_layout *lay,

@@ -20,9 +20,13 @@
 // contiguous range per persistent CTA. Item counts have a closed form, so each
 // CTA finds its range without a pre-pass.
 //
-// Roles: warp 0 issues TMA loads (keys: 64-row boxes, so a 128-key tile is two
-// loads, one per page in a paged cache; queries: one box per group), warp 1
-// allocates TMEM and issues the MMAs, the remaining warps run the epilogue.
+// Roles: four producer warps take every fourth tile and issue its TMA loads (keys
+// as two 64-row boxes, one per page in a paged cache, plus the keys' fp32 scales
+// by bulk copy; for a new query group also the group's query box and weights),
+// so several tiles are always being requested; one warp allocates TMEM and issues
+// the MMAs into one of several TMEM accumulators; eight warps run the epilogue
+// (decode: two groups of four take alternate tiles; prefill: all eight, two
+// query tokens each).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -39,14 +43,21 @@ template <int G>
 struct Cfg {
   static constexpr int N = kHI * G;
   static constexpr int kStages = G == 1 ? 8 : 4;
-  static constexpr int kEpiWarps = G == 1 ? 4 : 8;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kProdWarps = 4;                  // tile n is issued by producer warp n % 4
+  static constexpr int kMmaWarp = kProdWarps;
+  static constexpr int kEpiWarp0 = kProdWarps + 1;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kWarpsPerItem = G == 1 ? 4 : 8;  // decode: two groups of four warps alternate tiles
+  static constexpr int kAccBufs = G == 1 ? 8 : 2;       // TMEM accumulators (N columns each)
+  static constexpr int kThreads = 32 * (kProdWarps + 1 + kEpiWarps);
   static constexpr int kATile = kTileKeys * kDI;  // 16 KiB
   static constexpr int kBTile = N * kDI;          // 8 or 32 KiB
-  static constexpr int kTmemCols = 2 * N;         // two accumulator buffers (128 or 512)
-  static constexpr int kData = kStages * kATile + 2 * kBTile;
+  static constexpr int kWBytes = G * kHI * 4;     // head weights of a query group
+  static constexpr int kTmemCols = kAccBufs * N;  // 512
+  static constexpr int kData = kStages * kATile + 2 * kBTile + kStages * kTileKeys * 4 + 2 * kWBytes;
   static constexpr int kSmem = 1024 + kData + 1024;  // alignment slack + barriers
   static constexpr uint32_t kIdesc = instr_desc(0, 0, 0, 0, 128, N);
+  static_assert(kStages % kProdWarps == 0, "each producer warp owns whole stages");
 };
 
 struct Params {
@@ -54,6 +65,7 @@ struct Params {
   const float *k_scale;   // contiguous [B][n_max]; nullptr when paged
   const uint8_t *k_pool;  // paged pool base (scales live in the pages)
   const float *w;         // [T][64]
+  int scales_bulk;        // key scales reach shared memory by bulk copy (else read per thread)
   float *scores;          // [T][ld]
   long long ld;
   int T;
@@ -124,12 +136,13 @@ struct GroupMath {
   }
 };
 
-// A cursor over this CTA's items. All roles step identical cursors.
+// A cursor over this CTA's items (in order). Every role steps its own copy.
 template <int G>
 struct Cursor {
   int b, i, kt, ntiles, ng;
+  int gcount;      // query groups started so far in this CTA's range, the current one included
   SeqRows s;
-  long long left;  // items still to visit
+  long long left;  // items from the current one to the end of the range, the current one included
 
   __device__ void enter_seq(const Params &p, int nb) {
     b = nb;
@@ -148,13 +161,15 @@ struct Cursor {
     kt = (int)(f - GroupMath<G>::tiles_before(s, i));
     ntiles = GroupMath<G>::tiles_of(s, i);
     left = count;
+    gcount = 1;
   }
-  // advance; returns true when the next item starts a new group
+  // step one item; true when the new item starts a query group
   __device__ bool next(const Params &p) {
     --left;
     if (left <= 0) return false;
     if (++kt < ntiles) return false;
     kt = 0;
+    ++gcount;
     if (++i >= ng) {
       i = 0;
       do {
@@ -164,9 +179,62 @@ struct Cursor {
     ntiles = GroupMath<G>::tiles_of(s, i);
     return true;
   }
+  // step k >= 1 items
+  __device__ void advance(const Params &p, int k) {
+    if (kt + k < ntiles && left > k) {
+      kt += k;
+      left -= k;
+      return;
+    }
+    for (int j = 0; j < k; ++j) next(p);
+  }
   __device__ int row0() const { return s.r_lo + i * G; }
   __device__ int rows() const { return min(G, s.Qc - i * G); }
 };
+
+// One tile of a producer warp's 32-tile batch, held by the lane of the same index.
+struct Item {
+  int b, kt, row0;
+  int gslot;          // query group's B slot (0/1) | 2 if the tile starts the group | use count << 2
+  int pg0, pg1, has1;  // paged: physical pages of the tile's two 64-key halves
+};
+
+// Producer warp: walks the next (up to) 32 of its tiles — this warp's tiles are
+// every kProdWarps-th item — and has lane j keep tile j; for a paged cache each
+// lane starts loading its page ids. `n` is the item index of the cursor.
+template <int G>
+__device__ __forceinline__ int collect_batch(const Params &p, Cursor<G> &cur, long long &n, long long n_items,
+                                             int lane, Item &it) {
+  using C = Cfg<G>;
+  it.b = 0;
+  it.kt = 0;
+  it.row0 = 0;
+  it.gslot = 0;
+  it.pg0 = -1;
+  it.pg1 = -1;
+  it.has1 = 0;
+  int cnt = 0, len = 0;
+  for (int j = 0; j < 32 && n < n_items; ++j) {
+    if (lane == j) {
+      it.b = cur.b;
+      it.kt = cur.kt;
+      it.row0 = cur.row0();
+      const int g = cur.gcount - 1;
+      it.gslot = (g & 1) | ((cur.kt == 0 || n == 0) ? 2 : 0) | ((g >> 1) << 2);
+      len = cur.s.len;
+    }
+    ++cnt;
+    n += C::kProdWarps;
+    if (n < n_items) cur.advance(p, C::kProdWarps);
+  }
+  if (p.L.page_size && lane < cnt) {
+    const int *pt = p.L.page_table + (long long)it.b * p.L.max_pages + it.kt * 2;
+    it.pg0 = __ldg(pt);
+    it.has1 = it.kt * kTileKeys + 64 < len;
+    if (it.has1) it.pg1 = __ldg(pt + 1);
+  }
+  return cnt;
+}
 
 // ------------------------------------------------------------------ kernel
 template <int G>
@@ -179,15 +247,18 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   unsigned char *sA = base;
   unsigned char *sB = base + C::kStages * C::kATile;
+  float *sScale = reinterpret_cast<float *>(sB + 2 * C::kBTile);       // [stage][128] key scales
+  float *sW = sScale + C::kStages * kTileKeys;                         // [slot][G][64] head weights
   uint64_t *bars = reinterpret_cast<uint64_t *>(base + C::kData);
   uint64_t *a_full = bars, *a_empty = bars + C::kStages;
   uint64_t *b_full = bars + 2 * C::kStages, *b_empty = b_full + 2;
-  uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 2;
-  uint64_t *done_bar = acc_empty + 2;
+  uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + C::kAccBufs;
+  uint64_t *done_bar = acc_empty + C::kAccBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
   __shared__ long long s_range[2];  // first flat item of this CTA, number of items
   __shared__ int s_seq;             // sequence holding the first item
   __shared__ long long s_fseq;      // flat index of the first item within that sequence
+  __shared__ int s_b_turn;          // query-group loads issued so far (they are issued in group order)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.L.batch;
@@ -200,12 +271,11 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
     long long acc = 0;
     for (int b = b0; b < b1; ++b) {
-      const SeqRows s = seq_rows(p, b);
-      const long long n = GroupMath<G>::tiles_total(s);
+      const SeqRows sr = seq_rows(p, b);
+      const long long n = GroupMath<G>::tiles_total(sr);
       pre[b] = n;
       acc += n;
     }
-    // exclusive scan of thread totals
     long long incl = acc;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -236,12 +306,11 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     if (threadIdx.x == 0) {
       const long long f0 = W * blockIdx.x / gridDim.x;
       const long long f1 = W * (blockIdx.x + 1) / gridDim.x;
-      int lo = 0, hi = B - 1;  // last sequence with pre[b] <= f0 (and items)
+      int lo = 0, hi = B - 1;  // last sequence with pre[b] <= f0
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (pre[mid] <= f0) lo = mid; else hi = mid - 1;
       }
-      while (lo + 1 < B && pre[lo + 1] <= f0) ++lo;
       s_seq = lo;
       s_fseq = f0 - pre[lo];
       s_range[0] = f0;
@@ -253,20 +322,23 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
 
   // ---- barriers and TMEM
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(a_full + s, 1);
-      mbar_init(a_empty + s, 1);
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(a_full + st, 1);
+      mbar_init(a_empty + st, 1 + C::kWarpsPerItem);  // the MMA commit and the tile's epilogue warps
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(b_full + j, 1);
-      mbar_init(b_empty + j, 1);
+      mbar_init(b_empty + j, 1 + C::kEpiWarps);  // the MMA commit and every epilogue warp
+    }
+    for (int j = 0; j < C::kAccBufs; ++j) {
       mbar_init(acc_full + j, 1);
-      mbar_init(acc_empty + j, C::kEpiWarps);
+      mbar_init(acc_empty + j, C::kWarpsPerItem);
     }
     mbar_init(done_bar, 1);
+    s_b_turn = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::kMmaWarp) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -276,86 +348,124 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (n_items > 0) {
-    if (warp == 0) {
-      // ================= producer (one lane)
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
+    if (warp < C::kProdWarps) {
+      // ================= producer warps: tiles n with n % kProdWarps == warp
+      if (warp < n_items) {
+        if (lane == 0) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+        }
         Cursor<G> cur;
         cur.seek(p, s_seq, s_fseq, n_items);
-        int gcount = 0;
-        bool new_group = true;
-        uint32_t a_last_par[C::kStages];
-        bool a_used[C::kStages];
-        for (int s = 0; s < C::kStages; ++s) a_used[s] = false;
+        if (warp > 0) cur.advance(p, warp);
+        long long n_walk = warp;         // item the cursor is at
+        long long n_issue = warp;        // next item to issue
         bool ok = true;
-        for (long long n = 0; n < n_items && ok; ++n) {
-          if (new_group) {
-            const int slot = gcount & 1;
-            ok = mbar_wait(b_empty + slot, ((gcount >> 1) & 1) ^ 1, p.e, 0x410);
-            if (!ok) break;
-            mbar_expect_tx(b_full + slot, C::kBTile);
-            tma_load_2d(sB + slot * C::kBTile, &tm_q, b_full + slot, 0, cur.row0() * kHI);
-            ++gcount;
-          }
-          const int st = (int)(n % C::kStages);
-          const uint32_t use = (uint32_t)(n / C::kStages);
-          ok = mbar_wait(a_empty + st, (use & 1) ^ 1, p.e, 0x411);
-          if (!ok) break;
-          const int s0 = cur.kt * kTileKeys;
-          unsigned char *dst = sA + st * C::kATile;
-          int y0, y1 = -1;
-          if (p.L.page_size == 0) {
-            y0 = (int)((long long)cur.b * p.L.n_max + s0);
-            y1 = y0 + 64;
-          } else {
-            const int *pt = p.L.page_table + (long long)cur.b * p.L.max_pages;
-            const int pg0 = __ldg(pt + s0 / 64);
-            y0 = ((unsigned)pg0 < (unsigned)p.L.num_pages) ? pg0 * 66 : -1;
-            if (s0 + 64 < cur.s.len) {
-              const int pg1 = __ldg(pt + s0 / 64 + 1);
-              y1 = ((unsigned)pg1 < (unsigned)p.L.num_pages) ? pg1 * 66 : -2;
+        Item nxt;
+        int ncnt = collect_batch<G>(p, cur, n_walk, n_items, lane, nxt);
+        while (ncnt > 0 && ok) {
+          const Item it = nxt;
+          const int cnt = ncnt;
+          ncnt = n_walk < n_items ? collect_batch<G>(p, cur, n_walk, n_items, lane, nxt) : 0;
+          for (int j = 0; j < cnt; ++j, n_issue += C::kProdWarps) {
+            const int b = __shfl_sync(0xFFFFFFFFu, it.b, j);
+            const int kt = __shfl_sync(0xFFFFFFFFu, it.kt, j);
+            const int row0 = __shfl_sync(0xFFFFFFFFu, it.row0, j);
+            const int gs = __shfl_sync(0xFFFFFFFFu, it.gslot, j);
+            const int pg0 = __shfl_sync(0xFFFFFFFFu, it.pg0, j);
+            const int pg1 = __shfl_sync(0xFFFFFFFFu, it.pg1, j);
+            const int has1 = __shfl_sync(0xFFFFFFFFu, it.has1, j);
+            if (lane == 0) {
+              if (gs & 2) {  // first tile of a query group: its queries and weights
+                const int slot = gs & 1, use = gs >> 2;
+                // groups are loaded in order (one producer warp after another), so that
+                // each parity wait on a slot follows the wait for that slot's previous use
+                ok = wait_turn(&s_b_turn, use * 2 + slot, p.e, 0x415);
+                if (ok) ok = mbar_wait(b_empty + slot, (use & 1) ^ 1, p.e, 0x410);
+                if (ok) {
+                  const int nrow = min(G, p.T - row0);
+                  mbar_expect_tx(b_full + slot, C::kBTile + nrow * kHI * 4);
+                  tma_load_2d(sB + slot * C::kBTile, &tm_q, b_full + slot, 0, row0 * kHI);
+                  bulk_load(sW + slot * G * kHI, p.w + (long long)row0 * kHI, nrow * kHI * 4, b_full + slot);
+                  __threadfence_block();
+                  *reinterpret_cast<volatile int *>(&s_b_turn) = use * 2 + slot + 1;
+                }
+              }
+              const int st = (int)(n_issue % C::kStages);
+              const uint32_t use = (uint32_t)(n_issue / C::kStages);
+              if (ok) ok = mbar_wait(a_empty + st, (use & 1) ^ 1, p.e, 0x411);
+              if (ok) {
+                const int s0 = kt * kTileKeys;
+                unsigned char *dst = sA + st * C::kATile;
+                float *sdst = sScale + st * kTileKeys;
+                int y0 = -1, y1 = -1;
+                const unsigned char *sc0 = nullptr, *sc1 = nullptr;
+                uint32_t sb0 = 0, sb1 = 0;
+                if (p.L.page_size == 0) {
+                  y0 = (int)((long long)b * p.L.n_max + s0);
+                  y1 = y0 + 64;
+                  if (p.scales_bulk) {
+                    sc0 = reinterpret_cast<const unsigned char *>(p.k_scale + (long long)b * p.L.n_max + s0);
+                    sb0 = (uint32_t)min(kTileKeys, p.L.n_max - s0) * 4u;
+                  }
+                } else {
+                  const bool ok0 = (unsigned)pg0 < (unsigned)p.L.num_pages;
+                  const bool ok1 = has1 && (unsigned)pg1 < (unsigned)p.L.num_pages;
+                  if (!ok0 || (has1 && !ok1)) raise_error(p.e, DEV_BOUNDS, 0x412);
+                  if (ok0) {
+                    y0 = pg0 * 66;
+                    sc0 = p.k_pool + (long long)pg0 * 8448 + 8192;
+                    sb0 = 256;
+                  }
+                  if (ok1) {
+                    y1 = pg1 * 66;
+                    sc1 = p.k_pool + (long long)pg1 * 8448 + 8192;
+                    sb1 = 256;
+                  }
+                }
+                mbar_expect_tx(a_full + st, (y0 >= 0 ? 8192u : 0u) + (y1 >= 0 ? 8192u : 0u) + sb0 + sb1);
+                if (y0 >= 0) tma_load_2d(dst, &tm_k, a_full + st, 0, y0);
+                if (y1 >= 0) tma_load_2d(dst + 8192, &tm_k, a_full + st, 0, y1);
+                if (sb0) bulk_load(sdst, sc0, sb0, a_full + st);
+                if (sb1) bulk_load(sdst + 64, sc1, sb1, a_full + st);
+              }
             }
-            if (y0 == -1 || y1 == -2) raise_error(p.e, DEV_BOUNDS, 0x412);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+            if (!ok) break;
           }
-          const uint32_t bytes = (y0 >= 0 ? 8192u : 0u) + (y1 >= 0 ? 8192u : 0u);
-          mbar_expect_tx(a_full + st, bytes);
-          if (y0 >= 0) tma_load_2d(dst, &tm_k, a_full + st, 0, y0);
-          if (y1 >= 0) tma_load_2d(dst + 8192, &tm_k, a_full + st, 0, y1);
-          a_used[st] = true;
-          a_last_par[st] = use & 1;
-          new_group = cur.next(p);
         }
-        // make sure no copy is still landing in shared memory before exit
-        for (int s = 0; s < C::kStages; ++s)
-          if (a_used[s]) mbar_wait(a_full + s, a_last_par[s], p.e, 0x413);
-        for (int j = 0; j < 2 && j < gcount; ++j) {
-          const int last = gcount - 1 - j;  // the last use of each B slot
-          mbar_wait(b_full + (last & 1), (last >> 1) & 1, p.e, 0x414);
+        if (lane == 0) {
+          // no copy may still be landing in shared memory at exit: wait for the last
+          // tile this warp issued into each of its own stages (query slots: MMA warp)
+          const long long issued_end = n_issue;  // one past this warp's last issued item (stride kProdWarps)
+          for (int k = 1; k <= C::kStages / C::kProdWarps; ++k) {
+            const long long n_last = issued_end - (long long)k * C::kProdWarps;
+            if (n_last >= warp) mbar_wait(a_full + n_last % C::kStages, (uint32_t)(n_last / C::kStages) & 1, p.e, 0x413);
+          }
         }
       }
-    } else if (warp == 1) {
+      __syncwarp();
+    } else if (warp == C::kMmaWarp) {
       // ================= MMA issuer (one lane)
       if (lane == 0) {
         Cursor<G> cur;
         cur.seek(p, s_seq, s_fseq, n_items);
-        int gcount = 0;
         bool new_group = true;
         bool ok = true;
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         for (long long n = 0; n < n_items && ok; ++n) {
+          const int g = cur.gcount - 1;
+          const int slot = g & 1;
           if (new_group) {
-            ok = mbar_wait(b_full + (gcount & 1), (gcount >> 1) & 1, p.e, 0x420);
+            ok = mbar_wait(b_full + slot, (uint32_t)(g >> 1) & 1, p.e, 0x420);
             if (!ok) break;
-            ++gcount;
           }
-          const int slot = (gcount - 1) & 1;
           const int st = (int)(n % C::kStages);
           const uint32_t use = (uint32_t)(n / C::kStages);
-          const int ab = (int)(n & 1);
+          const int ab = (int)(n % C::kAccBufs);
           ok = mbar_wait(a_full + st, use & 1, p.e, 0x421);
           if (!ok) break;
-          ok = mbar_wait(acc_empty + ab, (((uint32_t)(n >> 1)) & 1) ^ 1, p.e, 0x422);
+          ok = mbar_wait(acc_empty + ab, ((uint32_t)(n / C::kAccBufs) & 1) ^ 1, p.e, 0x422);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(ab * C::N);
@@ -372,70 +482,108 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
         }
         umma_commit(done_bar);
         mbar_wait(done_bar, 0, p.e, 0x423);
+        // the query loads of the last two groups are the latest phases of the two slots
+        const int g_last = cur.gcount - 1;
+        for (int g = max(0, g_last - 1); g <= g_last; ++g) mbar_wait(b_full + (g & 1), (uint32_t)(g >> 1) & 1, p.e, 0x424);
       }
+      __syncwarp();
     } else {
       // ================= epilogue warps
-      const int ew = warp - 2;
+      const int ew = warp - C::kEpiWarp0;
       const int quad = warp & 3;         // TMEM lanes this warp may read
-      const int half = ew >> 2;          // G = 4: which pair of tokens
+      const int grp = ew >> 2;           // decode: tiles n with n % 2 == grp; prefill: token pair
       const int r = quad * 32 + lane;    // key row within the tile
       constexpr int kTokPerWarp = G == 1 ? 1 : 2;
       Cursor<G> cur;
       cur.seek(p, s_seq, s_fseq, n_items);
+      int g_seen = 0;                    // query groups whose weights this warp has checked in
+      float qs[kTokPerWarp];
+      for (int tt = 0; tt < kTokPerWarp; ++tt) qs[tt] = 0.f;
+      bool ok = true;
       for (long long n = 0; n < n_items; ++n) {
-        const int ab = (int)(n & 1);
-        if (!mbar_wait(acc_full + ab, ((uint32_t)(n >> 1)) & 1, p.e, 0x430)) break;
-        tc_fence_after();
-        const int s = cur.kt * kTileKeys + r;
-        const int b = cur.b;
-        // key scale
-        float sk = 0.f;
-        const bool key_ok = s < cur.s.len;
-        if (key_ok) {
-          if (p.L.page_size == 0) {
-            sk = __ldg(p.k_scale + (long long)b * p.L.n_max + s);
-          } else {
-            const int pg = __ldg(p.L.page_table + (long long)b * p.L.max_pages + s / 64);
-            if ((unsigned)pg < (unsigned)p.L.num_pages)
-              sk = __ldg(reinterpret_cast<const float *>(p.k_pool + (long long)pg * 8448 + 8192) + (s & 63));
-          }
-        }
-        const int nrows = cur.rows();
+        const int g = cur.gcount - 1;
+        const int slot = g & 1;
+        const bool mine = G != 1 || (int)(n & 1) == grp;
+        if (mine) {
+          if (g_seen <= g) {  // first tile of a group for this warp: its weights have landed
+            ok = mbar_wait(b_full + slot, (uint32_t)(g >> 1) & 1, p.e, 0x431);
+            if (!ok) break;
+            g_seen = g + 1;
 #pragma unroll
-        for (int tt = 0; tt < kTokPerWarp; ++tt) {
-          const int g = G == 1 ? 0 : half * 2 + tt;
-          uint32_t v[2][32];
-          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + g * kHI);
-          tmem_ld32(taddr, v[0]);
-          tmem_ld32(taddr + 32, v[1]);
-          const int t = cur.row0() + g;
-          const float4 *w4 = reinterpret_cast<const float4 *>(p.w + (long long)min(t, p.T - 1) * kHI);
-          tmem_ld_wait();
-          float acc = 0.f;
-#pragma unroll
-          for (int j4 = 0; j4 < kHI / 4; ++j4) {
-            const float4 wv = __ldg(w4 + j4);
-            const uint32_t *vv = v[j4 >> 3] + (j4 & 7) * 4;
-            acc = fmaf(wv.x, fmaxf(__uint_as_float(vv[0]), 0.f), acc);
-            acc = fmaf(wv.y, fmaxf(__uint_as_float(vv[1]), 0.f), acc);
-            acc = fmaf(wv.z, fmaxf(__uint_as_float(vv[2]), 0.f), acc);
-            acc = fmaf(wv.w, fmaxf(__uint_as_float(vv[3]), 0.f), acc);
+            for (int tt = 0; tt < kTokPerWarp; ++tt) {
+              const int t = cur.row0() + (G == 1 ? 0 : grp * 2 + tt);
+              qs[tt] = __ldg(p.q_scale + min(t, p.T - 1));
+            }
           }
-          const long long pos = cur.s.p_first + (long long)cur.i * G + g;
-          if (g < nrows && key_ok && s <= pos)
-            p.scores[(long long)t * p.ld + s] = acc * __ldg(p.q_scale + t) * sk;
+          const int ab = (int)(n % C::kAccBufs);
+          const int st = (int)(n % C::kStages);
+          ok = mbar_wait(acc_full + ab, (uint32_t)(n / C::kAccBufs) & 1, p.e, 0x430);
+          if (!ok) break;
+          tc_fence_after();
+          const int s = cur.kt * kTileKeys + r;
+          const int b = cur.b;
+          const bool key_ok = s < cur.s.len;
+          float sk = 0.f;
+          if (p.scales_bulk) {
+            sk = sScale[st * kTileKeys + r];
+          } else if (key_ok) {
+            if (p.L.page_size == 0) {
+              sk = __ldg(p.k_scale + (long long)b * p.L.n_max + s);
+            } else {
+              const int pg = __ldg(p.L.page_table + (long long)b * p.L.max_pages + s / 64);
+              if ((unsigned)pg < (unsigned)p.L.num_pages)
+                sk = __ldg(reinterpret_cast<const float *>(p.k_pool + (long long)pg * 8448 + 8192) + (s & 63));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_empty + st);  // keys and scales of this stage are no longer read here
+          const int nrows = cur.rows();
+#pragma unroll
+          for (int tt = 0; tt < kTokPerWarp; ++tt) {
+            const int gi = G == 1 ? 0 : grp * 2 + tt;
+            uint32_t v[2][32];
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + gi * kHI);
+            tmem_ld32(taddr, v[0]);
+            tmem_ld32(taddr + 32, v[1]);
+            const float4 *w4 = reinterpret_cast<const float4 *>(sW + (slot * G + gi) * kHI);
+            tmem_ld_wait();
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four independent chains
+#pragma unroll
+            for (int j4 = 0; j4 < kHI / 4; ++j4) {
+              const float4 wv = w4[j4];
+              const uint32_t *vv = v[j4 >> 3] + (j4 & 7) * 4;
+              a0 = fmaf(wv.x, fmaxf(__uint_as_float(vv[0]), 0.f), a0);
+              a1 = fmaf(wv.y, fmaxf(__uint_as_float(vv[1]), 0.f), a1);
+              a2 = fmaf(wv.z, fmaxf(__uint_as_float(vv[2]), 0.f), a2);
+              a3 = fmaf(wv.w, fmaxf(__uint_as_float(vv[3]), 0.f), a3);
+            }
+            const float acc = (a0 + a1) + (a2 + a3);
+            const long long pos = cur.s.p_first + (long long)cur.i * G + gi;
+            const int t = cur.row0() + gi;
+            if (gi < nrows && key_ok && s <= pos) p.scores[(long long)t * p.ld + s] = acc * qs[tt] * sk;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + ab);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty + ab);
-        cur.next(p);
+        const bool last = n + 1 == n_items;
+        const bool newg = cur.next(p);
+        if (newg || last) {  // this warp is done with group g: its query slot may be reloaded
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_empty + slot);
+        }
       }
     }
+  }
+  if (error_raised(p.e)) {
+    // a wait gave up somewhere: copies issued before that may still be in flight
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < 50000ull) __nanosleep(1000);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == C::kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // ------------------------------------------------------------------ host
@@ -497,6 +645,8 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
   p.k_pool = kI;
   p.w = w;
   p.scores = scores;
+  p.scales_bulk = L.page_size != 0 ||
+                  ((L.n_max % 4) == 0 && (reinterpret_cast<uintptr_t>(k_scale) & 15u) == 0);
   p.ld = ld;
   p.T = T;
   p.L = L;

@@ -3,12 +3,13 @@
 // selection paragraphs: K = 2048 tokens kept per query; openi.cn "DeepSeek-V3.2",
 // token-selection item).
 //
-// One thread-block cluster of C CTAs per row. Each CTA holds a contiguous
-// slice of the row in shared memory as order-preserving 32-bit keys, and the
-// cluster runs a 4-pass, 8-bit radix select of the k-th largest key with the
-// per-pass histograms summed over distributed shared memory. Selected
-// positions are then written in ascending position order: key > threshold, plus
-// the lowest-position ties at the threshold. The HBM row is read exactly once.
+// One thread-block cluster of C CTAs per row. Each CTA holds a contiguous slice
+// of the row in shared memory as order-preserving 32-bit keys. The cluster finds
+// the key of the k-th best score by radix select in three passes (11, 11 and 10
+// bits; the first histogram is built while loading), summing the per-CTA
+// histograms over distributed shared memory. Selected positions are then written
+// in ascending order: keys above the threshold plus the lowest-position keys equal
+// to it. The row is read from HBM exactly once.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -21,6 +22,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 1024;  // bits 31..21, 20..10, 9..0
 
 // Monotone map float -> uint32: larger float, larger key; -0 and +0 share a key;
 // every NaN maps below -inf.
@@ -32,14 +34,118 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 struct Shared {
-  unsigned hist[2][256];
-  unsigned total[256];
-  unsigned warp_gt[kWarps], warp_eq[kWarps];
+  unsigned hist1[kBins1], hist2[kBins2], hist3[kBins3];
+  unsigned wsum[kWarps];
+  unsigned wsum2[kWarps];
   unsigned cta_cnt[2];  // (greater, equal) counts of this CTA, read by the peers
-  unsigned prefix, mask, krem;
+  unsigned sel_bin, sel_krem;
   unsigned out_base, eq_take;
 };
 
+// Each thread holds the cluster-wide counts of W consecutive bins
+// [tid*W, tid*W + W). Finds, scanning from the highest bin down, the bin that
+// holds the krem-th largest key; stores it and the rank left inside it.
+template <int W>
+__device__ __forceinline__ void find_bin(const unsigned (&v)[W], unsigned krem, Shared &sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned s = 0;
+#pragma unroll
+  for (int i = 0; i < W; ++i) s += v[i];
+  unsigned incl = s;  // suffix sum over lanes >= lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned o = __shfl_down_sync(0xFFFFFFFFu, incl, off);
+    if (lane + off < 32) incl += o;
+  }
+  if (lane == 0) sm.wsum[warp] = incl;
+  __syncthreads();
+  unsigned above = incl - s;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w > warp) above += sm.wsum[w];
+  if (above < krem && krem <= above + s) {
+    unsigned c = above;
+#pragma unroll
+    for (int i = W - 1; i >= 0; --i) {
+      if (c + v[i] >= krem) {
+        sm.sel_bin = (unsigned)(tid * W + i);
+        sm.sel_krem = krem - c;
+        break;
+      }
+      c += v[i];
+    }
+  }
+  __syncthreads();
+}
+
+// Sum over the cluster of W consecutive bins per thread (all peers read at once).
+template <int C, int W>
+__device__ __forceinline__ void cluster_counts(cg::cluster_group &cluster, unsigned *h, unsigned (&v)[W]) {
+  const int tid = threadIdx.x;
+  unsigned peer[C][W];
+#pragma unroll
+  for (int r = 0; r < C; ++r) {
+    const unsigned *ph = cluster.map_shared_rank(h, r) + tid * W;
+    if (W == 4) {
+      const uint4 q = *reinterpret_cast<const uint4 *>(ph);
+      peer[r][0] = q.x;
+      peer[r][1 % W] = q.y;
+      peer[r][2 % W] = q.z;
+      peer[r][3 % W] = q.w;
+    } else {
+      const uint2 q = *reinterpret_cast<const uint2 *>(ph);
+      peer[r][0] = q.x;
+      peer[r][1 % W] = q.y;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < W; ++i) {
+    unsigned a = 0;
+#pragma unroll
+    for (int r = 0; r < C; ++r) a += peer[r][i];
+    v[i] = a;
+  }
+}
+
+// Exclusive prefix over the block of a per-thread pair (a, b); returns the
+// block totals through the references.
+__device__ __forceinline__ void block_scan2(unsigned &a, unsigned &b, unsigned &tot_a, unsigned &tot_b,
+                                            Shared &sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned oa = __shfl_up_sync(0xFFFFFFFFu, ia, off);
+    const unsigned ob = __shfl_up_sync(0xFFFFFFFFu, ib, off);
+    if (lane >= off) {
+      ia += oa;
+      ib += ob;
+    }
+  }
+  if (lane == 31) {
+    sm.wsum[warp] = ia;
+    sm.wsum2[warp] = ib;
+  }
+  __syncthreads();
+  unsigned pa = 0, pb = 0, ta = 0, tb = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const unsigned x = sm.wsum[w], y = sm.wsum2[w];
+    if (w < warp) {
+      pa += x;
+      pb += y;
+    }
+    ta += x;
+    tb += y;
+  }
+  a = pa + ia - a;
+  b = pb + ib - b;
+  tot_a = ta;
+  tot_b = tb;
+  __syncthreads();
+}
+
+template <int C>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict__ scores, long long ld, int k,
                                                         Layout L, int cap, int *__restrict__ idx, ErrCtx e) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -47,10 +153,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + ((sizeof(Shared) + 15) & ~size_t(15)));
 
   cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int t = blockIdx.x / C;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
 
   const RowPos rp = row_position(L, t);
   long long n = (long long)rp.pos + 1;
@@ -68,170 +173,152 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
     return;  // no distributed shared memory was touched
   }
 
-  // ---- this CTA's slice of the row, as keys in shared memory
+  for (int i = tid; i < kBins1; i += kThreads) sm.hist1[i] = 0;
+  for (int i = tid; i < kBins2; i += kThreads) sm.hist2[i] = 0;
+  for (int i = tid; i < kBins3; i += kThreads) sm.hist3[i] = 0;
+  __syncthreads();
+
+  // ---- this CTA's slice as keys in shared memory; histogram of bits 31..21
   const int chunk = (int)((((n + C - 1) / C) + 31) / 32 * 32);
   const long long lo = (long long)rank * chunk;
   const int cnt = (int)max(0LL, min(n, lo + chunk) - lo);
-  const float *row = scores + (long long)t * ld + lo;
   {
+    const float *row = scores + (long long)t * ld + lo;
     const int n4 = cnt >> 2;
     const float4 *r4 = reinterpret_cast<const float4 *>(row);
-    for (int i = tid; i < n4; i += kThreads) {
-      float4 v = __ldcs(r4 + i);
-      uint4 kk = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
-      reinterpret_cast<uint4 *>(keys)[i] = kk;
-    }
-    for (int i = (n4 << 2) + tid; i < cnt; i += kThreads) keys[i] = order_key(__ldcs(row + i));
-  }
-  if (tid == 0) {
-    sm.prefix = 0;
-    sm.mask = 0;
-    sm.krem = (unsigned)k;
-  }
-
-  // contiguous per-warp segments (multiples of 32) keep lanes converged
-  const int seg = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-  const int wlo = warp * seg;
-
-  // ---- radix select of the k-th largest key, 8 bits per pass
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    unsigned *h = sm.hist[pass & 1];
-    for (int i = tid; i < 256; i += kThreads) h[i] = 0;
-    __syncthreads();
-    const unsigned prefix = sm.prefix, mask = sm.mask;
-    for (int j = lane; j < seg; j += 32) {
-      const int i = wlo + j;
-      int bin = -1;
-      if (i < cnt) {
-        const uint32_t key = keys[i];
-        if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
-      }
-      const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
-      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&h[bin], (unsigned)__popc(peers));
-    }
-    cluster.sync();
-    if (tid < 256) {
-      unsigned s = 0;
-      for (int r = 0; r < C; ++r) s += cluster.map_shared_rank(h, r)[tid];
-      sm.total[tid] = s;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const unsigned krem = sm.krem;
-      unsigned v[8], s = 0;
+    constexpr int U = 8;  // float4 loads in flight per thread
+    for (int base = 0; base < n4; base += U * kThreads) {
+      float4 v[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[i] = sm.total[lane * 8 + i];
-        s += v[i];
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * kThreads + tid;
+        if (i < n4) v[u] = __ldcs(r4 + i);
       }
-      unsigned suf = s;  // inclusive suffix sum over lanes
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const unsigned o = __shfl_down_sync(0xFFFFFFFFu, suf, off);
-        if (lane + off < 32) suf += o;
-      }
-      const unsigned above = suf - s;
-      if (above < krem && krem <= suf) {
-        unsigned c = above;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (c + v[i] >= krem) {
-            sm.prefix = prefix | ((unsigned)(lane * 8 + i) << shift);
-            sm.mask = mask | (255u << shift);
-            sm.krem = krem - c;
-            break;
-          }
-          c += v[i];
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * kThreads + tid;
+        if (i < n4) {
+          const uint4 kk = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
+          reinterpret_cast<uint4 *>(keys)[i] = kk;
+          atomicAdd(sm.hist1 + (kk.x >> 21), 1u);
+          atomicAdd(sm.hist1 + (kk.y >> 21), 1u);
+          atomicAdd(sm.hist1 + (kk.z >> 21), 1u);
+          atomicAdd(sm.hist1 + (kk.w >> 21), 1u);
         }
       }
     }
-    __syncthreads();
+    const int i = (n4 << 2) + tid;  // 0..3 trailing keys
+    if (i < cnt) {
+      const uint32_t kx = order_key(__ldcs(row + i));
+      keys[i] = kx;
+      atomicAdd(sm.hist1 + (kx >> 21), 1u);
+    }
   }
-  const uint32_t thr = sm.prefix;
-  const unsigned krem = sm.krem;  // ties at the threshold still to take
 
-  // ---- counts per warp, per CTA, then across the cluster
+  // ---- pass 1: bits 31..21
+  cluster.sync();
+  unsigned krem = (unsigned)k;
+  uint32_t prefix;
   {
-    unsigned gt = 0, eq = 0;
-    for (int j = lane; j < seg; j += 32) {
-      const int i = wlo + j;
-      const uint32_t key = i < cnt ? keys[i] : 0u;
-      const bool in = i < cnt;
-      gt += __popc(__ballot_sync(0xFFFFFFFFu, in && key > thr));
-      eq += __popc(__ballot_sync(0xFFFFFFFFu, in && key == thr));
-    }
-    if (lane == 0) {
-      sm.warp_gt[warp] = gt;
-      sm.warp_eq[warp] = eq;
-    }
+    unsigned v[4];
+    cluster_counts<C, 4>(cluster, sm.hist1, v);
+    find_bin<4>(v, krem, sm);
+    prefix = sm.sel_bin;  // top 11 bits
+    krem = sm.sel_krem;
   }
-  __syncthreads();
+  // ---- pass 2: bits 20..10 among keys whose top 11 bits match
+#pragma unroll 4
+  for (int i = tid; i < cnt; i += kThreads) {
+    const uint32_t key = keys[i];
+    if ((key >> 21) == prefix) atomicAdd(sm.hist2 + ((key >> 10) & 2047u), 1u);
+  }
+  cluster.sync();
+  {
+    unsigned v[4];
+    cluster_counts<C, 4>(cluster, sm.hist2, v);
+    find_bin<4>(v, krem, sm);
+    prefix = (prefix << 11) | sm.sel_bin;  // top 22 bits
+    krem = sm.sel_krem;
+  }
+  // ---- pass 3: bits 9..0 among keys whose top 22 bits match
+#pragma unroll 4
+  for (int i = tid; i < cnt; i += kThreads) {
+    const uint32_t key = keys[i];
+    if ((key >> 10) == prefix) atomicAdd(sm.hist3 + (key & 1023u), 1u);
+  }
+  cluster.sync();
+  {
+    unsigned v[2];
+    cluster_counts<C, 2>(cluster, sm.hist3, v);
+    find_bin<2>(v, krem, sm);
+    prefix = (prefix << 10) | sm.sel_bin;  // the threshold key
+    krem = sm.sel_krem;                    // keys equal to it still to take
+  }
+  const uint32_t thr = prefix;
+
+  // ---- each thread owns a contiguous run of the slice: counts, block scan, cluster scan
+  const int run = (cnt + kThreads - 1) / kThreads;
+  const int r0 = min(cnt, tid * run), r1 = min(cnt, r0 + run);
+  unsigned gt = 0, eq = 0;
+  for (int i = r0; i < r1; ++i) {
+    const uint32_t key = keys[i];
+    gt += key > thr;
+    eq += key == thr;
+  }
+  unsigned cta_gt, cta_eq;
+  block_scan2(gt, eq, cta_gt, cta_eq, sm);  // gt, eq now exclusive prefixes within the CTA
   if (tid == 0) {
-    unsigned g = 0, q = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const unsigned a = sm.warp_gt[w], b = sm.warp_eq[w];
-      sm.warp_gt[w] = g;  // exclusive prefixes
-      sm.warp_eq[w] = q;
-      g += a;
-      q += b;
-    }
-    sm.cta_cnt[0] = g;
-    sm.cta_cnt[1] = q;
+    sm.cta_cnt[0] = cta_gt;
+    sm.cta_cnt[1] = cta_eq;
   }
   cluster.sync();
   if (tid == 0) {
-    unsigned gt_before = 0, eq_before = 0;
-    for (int r = 0; r < rank; ++r) {
-      const unsigned *pc = cluster.map_shared_rank(sm.cta_cnt, r);
-      gt_before += pc[0];
-      eq_before += pc[1];
+    unsigned pc[C][2];
+#pragma unroll
+    for (int r = 0; r < C; ++r) {
+      const uint2 c2 = *reinterpret_cast<const uint2 *>(cluster.map_shared_rank(sm.cta_cnt, r));
+      pc[r][0] = c2.x;
+      pc[r][1] = c2.y;
     }
-    const unsigned mine = sm.cta_cnt[1];
+    unsigned gt_before = 0, eq_before = 0;
+#pragma unroll
+    for (int r = 0; r < C; ++r)
+      if (r < rank) {
+        gt_before += pc[r][0];
+        eq_before += pc[r][1];
+      }
     const unsigned taken_before = min(eq_before, krem);
-    sm.eq_take = min(mine, krem - taken_before);
+    sm.eq_take = min(cta_eq, krem - taken_before);
     sm.out_base = gt_before + taken_before;
   }
   cluster.sync();  // peers are done reading this CTA's counts after this point
 
-  // ---- emit selected positions in ascending order
+  // ---- emit this thread's selected positions in ascending order
   {
     const unsigned eq_take = sm.eq_take;
-    const unsigned eq_pre = sm.warp_eq[warp];
-    unsigned base = sm.out_base + sm.warp_gt[warp] + min(eq_pre, eq_take);
-    unsigned tie = eq_pre;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int j = lane; j < seg; j += 32) {
-      const int i = wlo + j;
-      const bool in = i < cnt;
-      const uint32_t key = in ? keys[i] : 0u;
-      const bool is_eq = in && key == thr;
-      const unsigned eqm = __ballot_sync(0xFFFFFFFFu, is_eq);
-      const bool take = (in && key > thr) || (is_eq && tie + __popc(eqm & lt) < eq_take);
-      const unsigned selm = __ballot_sync(0xFFFFFFFFu, take);
-      if (take) {
-        const unsigned p = base + __popc(selm & lt);
-        if (p < (unsigned)k) out[p] = (int)(lo + i);
+    unsigned tie = eq;                                  // ties before this thread's run
+    unsigned o = sm.out_base + gt + min(eq, eq_take);   // selected before this thread's run
+    for (int i = r0; i < r1; ++i) {
+      const uint32_t key = keys[i];
+      bool take = key > thr;
+      if (key == thr) {
+        take = tie < eq_take;
+        ++tie;
       }
-      base += __popc(selm);
-      tie += __popc(eqm);
+      if (take) {
+        if (o < (unsigned)k) out[o] = (int)(lo + i);
+        ++o;
+      }
     }
   }
 }
 
-}  // namespace
-
-size_t topk_smem_bytes(int cap) { return ((sizeof(Shared) + 15) & ~size_t(15)) + (size_t)cap * 4; }
-
-cudaError_t launch_topk(const float *scores, long long ld, int T, int k, const Layout &L, int C, int cap, int *idx,
-                        const ErrCtx &e, cudaStream_t stream) {
+template <int C>
+cudaError_t launch_c(const float *scores, long long ld, int T, int k, const Layout &L, int cap, int *idx,
+                     const ErrCtx &e, cudaStream_t stream) {
   const size_t smem = topk_smem_bytes(cap);
-  cudaError_t err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = cudaFuncSetAttribute(topk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  if (C > 8) {
-    err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (err != cudaSuccess) return err;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)T * C);
   cfg.blockDim = dim3(kThreads);
@@ -244,7 +331,22 @@ cudaError_t launch_topk(const float *scores, long long ld, int T, int k, const L
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, k, L, cap, idx, e);
+  return cudaLaunchKernelEx(&cfg, topk_kernel<C>, scores, ld, k, L, cap, idx, e);
+}
+
+}  // namespace
+
+size_t topk_smem_bytes(int cap) { return ((sizeof(Shared) + 15) & ~size_t(15)) + (size_t)cap * 4; }
+
+cudaError_t launch_topk(const float *scores, long long ld, int T, int k, const Layout &L, int C, int cap, int *idx,
+                        const ErrCtx &e, cudaStream_t stream) {
+  switch (C) {
+    case 1: return launch_c<1>(scores, ld, T, k, L, cap, idx, e, stream);
+    case 2: return launch_c<2>(scores, ld, T, k, L, cap, idx, e, stream);
+    case 4: return launch_c<4>(scores, ld, T, k, L, cap, idx, e, stream);
+    case 8: return launch_c<8>(scores, ld, T, k, L, cap, idx, e, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dsa

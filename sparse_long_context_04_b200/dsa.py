@@ -56,7 +56,7 @@ _lib = None
 
 EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size", "dsa_sparse_mqa_attn",
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
-           "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc")
+           "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site")
 
 
 def lib() -> ctypes.CDLL:
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_forward_workspace_size.restype = sz
         L.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
         L.dsa_get_device_error.argtypes = [vp]
+        L.dsa_get_device_error_site.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        L.dsa_get_device_error_site.restype = i
         L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.dsa_status_string.argtypes = [i]
         L.dsa_status_string.restype = ctypes.c_char_p
@@ -211,6 +213,13 @@ def dsa_forward(args: ForwardArgs, workspace, stream=None):
 
 def dsa_get_device_error(stream=None) -> int:
     return int(lib().dsa_get_device_error(_stream(stream)))
+
+
+def dsa_get_device_error_site(stream=None):
+    """(status, site code of the first failing device check or wait)."""
+    site = ctypes.c_uint(0)
+    st = int(lib().dsa_get_device_error_site(_stream(stream), ctypes.byref(site)))
+    return st, int(site.value)
 
 
 def dsa_set_wait_limit_ns(ns: int):
