@@ -23,10 +23,11 @@
 // Roles: four producer warps take every fourth tile and issue its TMA loads (keys
 // as two 64-row boxes, one per page in a paged cache, plus the keys' fp32 scales
 // by bulk copy; for a new query group also the group's query box and weights),
-// so several tiles are always being requested; one warp allocates TMEM and issues
-// the MMAs into one of several TMEM accumulators; eight warps run the epilogue
-// (decode: two groups of four take alternate tiles; prefill: all eight, two
-// query tokens each).
+// so several tiles are always being requested; two MMA warps take alternate tiles
+// and issue their MMAs into separate TMEM accumulators (one issuing thread cannot
+// keep up with HBM: each tile needs waits, four MMAs and two commits); eight warps
+// run the epilogue (decode: two groups of four take alternate tiles; prefill: all
+// eight, two query tokens each).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -44,12 +45,13 @@ struct Cfg {
   static constexpr int N = kHI * G;
   static constexpr int kStages = G == 1 ? 8 : 4;
   static constexpr int kProdWarps = 4;                  // tile n is issued by producer warp n % 4
-  static constexpr int kMmaWarp = kProdWarps;
-  static constexpr int kEpiWarp0 = kProdWarps + 1;
+  static constexpr int kMmaWarps = 2;                   // tile n's MMAs are issued by MMA warp n % 2
+  static constexpr int kMmaWarp0 = kProdWarps;
+  static constexpr int kEpiWarp0 = kProdWarps + kMmaWarps;
   static constexpr int kEpiWarps = 8;
   static constexpr int kWarpsPerItem = G == 1 ? 4 : 8;  // decode: two groups of four warps alternate tiles
   static constexpr int kAccBufs = G == 1 ? 8 : 2;       // TMEM accumulators (N columns each)
-  static constexpr int kThreads = 32 * (kProdWarps + 1 + kEpiWarps);
+  static constexpr int kThreads = 32 * (kProdWarps + kMmaWarps + kEpiWarps);
   static constexpr int kATile = kTileKeys * kDI;  // 16 KiB
   static constexpr int kBTile = N * kDI;          // 8 or 32 KiB
   static constexpr int kWBytes = G * kHI * 4;     // head weights of a query group
@@ -253,8 +255,8 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   uint64_t *a_full = bars, *a_empty = bars + C::kStages;
   uint64_t *b_full = bars + 2 * C::kStages, *b_empty = b_full + 2;
   uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + C::kAccBufs;
-  uint64_t *done_bar = acc_empty + C::kAccBufs;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+  uint64_t *done_bar = acc_empty + C::kAccBufs;  // one per MMA warp
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + C::kMmaWarps);
   __shared__ long long s_range[2];  // first flat item of this CTA, number of items
   __shared__ int s_seq;             // sequence holding the first item
   __shared__ long long s_fseq;      // flat index of the first item within that sequence
@@ -328,17 +330,17 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(b_full + j, 1);
-      mbar_init(b_empty + j, 1 + C::kEpiWarps);  // the MMA commit and every epilogue warp
+      mbar_init(b_empty + j, C::kMmaWarps + C::kEpiWarps);  // every MMA and epilogue warp
     }
     for (int j = 0; j < C::kAccBufs; ++j) {
       mbar_init(acc_full + j, 1);
       mbar_init(acc_empty + j, C::kWarpsPerItem);
     }
-    mbar_init(done_bar, 1);
+    for (int j = 0; j < C::kMmaWarps; ++j) mbar_init(done_bar + j, 1);
     s_b_turn = 0;
     fence_mbar_init();
   }
-  if (warp == C::kMmaWarp) {
+  if (warp == C::kMmaWarp0) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -445,46 +447,53 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
         }
       }
       __syncwarp();
-    } else if (warp == C::kMmaWarp) {
-      // ================= MMA issuer (one lane)
+    } else if (warp < C::kEpiWarp0) {
+      // ================= MMA warps (one lane each): tiles n with n % kMmaWarps == mw
+      const int mw = warp - C::kMmaWarp0;
       if (lane == 0) {
         Cursor<G> cur;
         cur.seek(p, s_seq, s_fseq, n_items);
-        bool new_group = true;
+        int g_seen = 0;  // query groups whose slot this warp has waited for
         bool ok = true;
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         for (long long n = 0; n < n_items && ok; ++n) {
           const int g = cur.gcount - 1;
           const int slot = g & 1;
-          if (new_group) {
-            ok = mbar_wait(b_full + slot, (uint32_t)(g >> 1) & 1, p.e, 0x420);
+          if ((int)(n % C::kMmaWarps) == mw) {
+            if (g_seen <= g) {
+              ok = mbar_wait(b_full + slot, (uint32_t)(g >> 1) & 1, p.e, 0x420);
+              if (!ok) break;
+              g_seen = g + 1;
+            }
+            const int st = (int)(n % C::kStages);
+            const uint32_t use = (uint32_t)(n / C::kStages);
+            const int ab = (int)(n % C::kAccBufs);
+            ok = mbar_wait(a_full + st, use & 1, p.e, 0x421);
             if (!ok) break;
-          }
-          const int st = (int)(n % C::kStages);
-          const uint32_t use = (uint32_t)(n / C::kStages);
-          const int ab = (int)(n % C::kAccBufs);
-          ok = mbar_wait(a_full + st, use & 1, p.e, 0x421);
-          if (!ok) break;
-          ok = mbar_wait(acc_empty + ab, ((uint32_t)(n / C::kAccBufs) & 1) ^ 1, p.e, 0x422);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(ab * C::N);
+            ok = mbar_wait(acc_empty + ab, ((uint32_t)(n / C::kAccBufs) & 1) ^ 1, p.e, 0x422);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)(ab * C::N);
 #pragma unroll
-          for (int ks = 0; ks < kDI / 32; ++ks) {
-            const uint64_t ad = smem_desc(a0 + st * C::kATile + ks * 32, 16, 1024, SW_128B);
-            const uint64_t bd = smem_desc(b0 + slot * C::kBTile + ks * 32, 16, 1024, SW_128B);
-            umma_f8(d, ad, bd, C::kIdesc, ks > 0);
+            for (int ks = 0; ks < kDI / 32; ++ks) {
+              const uint64_t ad = smem_desc(a0 + st * C::kATile + ks * 32, 16, 1024, SW_128B);
+              const uint64_t bd = smem_desc(b0 + slot * C::kBTile + ks * 32, 16, 1024, SW_128B);
+              umma_f8(d, ad, bd, C::kIdesc, ks > 0);
+            }
+            umma_commit(a_empty + st);
+            umma_commit(acc_full + ab);
           }
-          umma_commit(a_empty + st);
-          umma_commit(acc_full + ab);
-          new_group = cur.next(p);
-          if (new_group || n + 1 == n_items) umma_commit(b_empty + slot);
+          // leaving group g: this warp's MMAs on the group's query slot are issued
+          if (cur.next(p) || n + 1 == n_items) umma_commit(b_empty + slot);
         }
-        umma_commit(done_bar);
-        mbar_wait(done_bar, 0, p.e, 0x423);
-        // the query loads of the last two groups are the latest phases of the two slots
-        const int g_last = cur.gcount - 1;
-        for (int g = max(0, g_last - 1); g <= g_last; ++g) mbar_wait(b_full + (g & 1), (uint32_t)(g >> 1) & 1, p.e, 0x424);
+        umma_commit(done_bar + mw);
+        mbar_wait(done_bar + mw, 0, p.e, 0x423);
+        if (mw == 0) {
+          // the query loads of the last two groups are the latest phases of the two slots
+          const int g_last = cur.gcount - 1;
+          for (int g = max(0, g_last - 1); g <= g_last; ++g)
+            mbar_wait(b_full + (g & 1), (uint32_t)(g >> 1) & 1, p.e, 0x424);
+        }
       }
       __syncwarp();
     } else {
@@ -583,7 +592,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == C::kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == C::kMmaWarp0) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // ------------------------------------------------------------------ host
