@@ -35,14 +35,18 @@ constexpr int kStages = 3;
 constexpr int kQTile = kH * 128;               // 16 KiB
 constexpr int kKTile = kMaxKeys * 128;         // 32 KiB
 constexpr int kStage = kQTile + kKTile;        // 48 KiB
-constexpr int kRing = kStages * kStage;        // 144 KiB (also holds two 64 KiB value blocks)
-constexpr int kVBlock = 64 * kDv * 2;          // 64 KiB: 64 rows x 512 values
+constexpr int kRing = kStages * kStage;        // 144 KiB (later: four 32 KiB value blocks)
+constexpr int kVKeys = 32;                     // value rows per block
+constexpr int kVBlock = kVKeys * kDv * 2;      // 32 KiB
+constexpr int kVStages = 4;
 constexpr int kPBytes = kH * kMaxKeys * 2;     // 64 KiB
 constexpr int kProducers = 128;                // warps 0-3
 constexpr int kMmaWarp = 4;
-constexpr int kThreads = 288;                  // + MMA warp + 4 softmax warps
+constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per TMEM lane quadrant
+constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
 constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 8 + 256 + 1024;
 constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
+static_assert(kVStages * kVBlock <= kRing, "value blocks reuse the score ring");
 
 struct Params {
   const __nv_bfloat16 *kv;
@@ -52,7 +56,7 @@ struct Params {
   int keys_per_split;
   float scale_log2;   // softmax_scale * log2(e)
   float scale;
-  float *o_part;      // [rows][splits][128][512]
+  float *o_part;      // [rows][splits][512 values][128 heads] (head-minor: coalesced stores)
   float2 *ml_part;    // [rows][splits][128]: (max * scale, sum)
   Layout L;
   ErrCtx e;
@@ -62,6 +66,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&v);
 }
+
+// the eight softmax/output warps only
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
@@ -73,11 +80,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long *rows = reinterpret_cast<long long *>(sP + kPBytes);
   uint64_t *bars = reinterpret_cast<uint64_t *>(rows + kMaxKeys);
   uint64_t *full = bars, *empty = bars + kStages;
-  uint64_t *vfull = bars + 2 * kStages, *vempty = vfull + 2;
-  uint64_t *s_full = vempty + 2, *p_full = s_full + 1, *o_full = p_full + 1;
+  uint64_t *vfull = bars + 2 * kStages, *vempty = vfull + kVStages;
+  uint64_t *s_full = vempty + kVStages, *p_full = s_full + 1, *o_full = p_full + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
   __shared__ int s_nvalid;
   __shared__ uint32_t s_valid[kMaxKeys / 32];  // bit i: selected entry i is a real row
+  __shared__ float s_part[2][kH];              // per-half row max, then row sum
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x / p.splits;     // row within this launch
@@ -86,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = min(p.keys_per_split, p.k - k0);
   const long long part = (long long)t * p.splits + split;
 
-  // ---- selected rows of this split (top-k output: valid positions first, then -1)
+  // ---- selected rows of this split (-1 entries are padding, anywhere in the list)
   if (threadIdx.x == 0) s_nvalid = 0;
   if (threadIdx.x < kMaxKeys / 32) s_valid[threadIdx.x] = 0;
   __syncthreads();
@@ -113,20 +121,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x < kH) p.ml_part[part * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
     return;
   }
-  const int nkb = (nvalid + 63) / 64;  // 64-key blocks
-  const int n = nkb * 64;              // MMA N of the score tile
+  const int n = ((nvalid + 63) / 64) * 64;  // MMA N of the score tile
+  const int nvb = (nvalid + kVKeys - 1) / kVKeys;  // value blocks
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full + s, kProducers + 1);
       mbar_init(empty + s, 1);
     }
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < kVStages; ++j) {
       mbar_init(vfull + j, kProducers);
       mbar_init(vempty + j, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, kSmWarps);
     mbar_init(o_full, 1);
     fence_mbar_init();
   }
@@ -165,16 +173,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // value rows: wait until every score MMA has consumed the ring
     if (ok) ok = mbar_wait(s_full, 0, p.e, 0x511);
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int st = kb & 1;
-      ok = mbar_wait(vempty + st, ((kb >> 1) & 1) ^ 1, p.e, 0x512);
+    for (int vb = 0; vb < nvb && ok; ++vb) {
+      const int st = vb % kVStages;
+      ok = mbar_wait(vempty + st, ((vb / kVStages) & 1) ^ 1, p.e, 0x512);
       if (!ok) break;
       const uint32_t sv = smem_u32(ring + st * kVBlock);
-      for (int q = tid; q < 64 * 64; q += kProducers) {
+      for (int q = tid; q < kVKeys * 64; q += kProducers) {
         const int i = q >> 6, u = q & 63;
-        const long long r = rows[kb * 64 + i];
+        const long long r = rows[vb * kVKeys + i];
         const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + u * 16;
-        cp_async16_zfill(sv + (u >> 3) * 8192 + sw128_off(i, u & 7), src, r >= 0);
+        cp_async16_zfill(sv + (u >> 3) * (kVKeys * 128) + sw128_off(i, u & 7), src, r >= 0);
       }
       cp_async_arrive_noinc(vfull + st);
     }
@@ -201,19 +209,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(s_full);
       if (ok) ok = mbar_wait(p_full, 0, p.e, 0x521);
       if (ok) tc_fence_after();
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int st = kb & 1;
-        ok = mbar_wait(vfull + st, (kb >> 1) & 1, p.e, 0x522);
+      for (int vb = 0; vb < nvb && ok; ++vb) {
+        const int st = vb % kVStages;
+        ok = mbar_wait(vfull + st, (vb / kVStages) & 1, p.e, 0x522);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t va = r0 + st * kVBlock, pa = p0 + kb * 16384;
+        // value rows vb*32 .. +31: their P columns sit in 64-key block vb/2, bytes (vb%2)*64 of each row
+        const uint32_t va = r0 + st * kVBlock, pa = p0 + (vb >> 1) * 16384 + (vb & 1) * 64;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
+        for (int ks = 0; ks < kVKeys / 16; ++ks) {
           const uint64_t ad = smem_desc(pa + ks * 32, 16, 1024, SW_128B);
 #pragma unroll
           for (int nh = 0; nh < 2; ++nh)
-            umma_f16(tmem + nh * 256, ad, smem_desc(va + nh * 4 * 8192 + ks * 2048, 8192, 1024, SW_128B),
-                     idesc_pv, (kb | ks) != 0);
+            umma_f16(tmem + nh * 256, ad,
+                     smem_desc(va + nh * 4 * (kVKeys * 128) + ks * 2048, kVKeys * 128, 1024, SW_128B), idesc_pv,
+                     (vb | ks) != 0);
         }
         umma_commit(vempty + st);
       }
@@ -221,25 +231,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ================= softmax + output (warps 5..8, one head row per thread)
+    // ================= softmax + output: 8 warps, two per TMEM lane quadrant, each half the columns
+    const int sw = warp - kSmWarp0;
     const int quad = warp & 3;
+    const int half = sw >> 2;
     const int h = quad * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const int j0 = half * (n / 64), j1 = j0 + n / 64;  // this half's 32-column chunks
     float m = -INFINITY, l = 0.f;
     bool ok = mbar_wait(s_full, 0, p.e, 0x530);
     if (ok) {
       tc_fence_after();
-      for (int j = 0; j < n / 32; ++j) {
-        uint32_t v[32];
-        tmem_ld32(trow + j * 32, v);
+      for (int j = j0; j < j1; j += 2) {  // two TMEM loads per wait
+        uint32_t v[2][32];
+        tmem_ld32(trow + j * 32, v[0]);
+        if (j + 1 < j1) tmem_ld32(trow + (j + 1) * 32, v[1]);
         tmem_ld_wait();
-        const uint32_t vm = s_valid[j];
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if ((vm >> x) & 1u) m = fmaxf(m, __uint_as_float(v[x]));
+        for (int u = 0; u < 2; ++u) {
+          if (j + u >= j1) break;
+          const uint32_t vm = s_valid[j + u];
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if ((vm >> x) & 1u) m = fmaxf(m, __uint_as_float(v[u][x]));
+        }
       }
-      const float mb = m * p.scale_log2;
-      for (int j = 0; j < n / 32; ++j) {
+    }
+    s_part[half][h] = m;
+    softmax_bar();
+    m = fmaxf(s_part[0][h], s_part[1][h]);
+    softmax_bar();  // both halves have read the maxima
+    const float mb = m * p.scale_log2;
+    if (ok) {
+      for (int j = j0; j < j1; ++j) {
         uint32_t v[32];
         tmem_ld32(trow + j * 32, v);
         tmem_ld_wait();
@@ -266,23 +290,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      ok = mbar_wait(o_full, 0, p.e, 0x531);
     }
+    s_part[half][h] = l;
+    softmax_bar();
+    l = s_part[0][h] + s_part[1][h];
+    if (ok) ok = mbar_wait(o_full, 0, p.e, 0x531);
     if (ok) {
       tc_fence_after();
-      float *orow = p.o_part + (part * kH + h) * kDv;
-      for (int j = 0; j < kDv / 32; ++j) {
-        uint32_t v[32];
-        tmem_ld32(trow + j * 32, v);
+      // this warp's 256 output columns; stores are head-minor so each warp writes whole lines
+      float *ob = p.o_part + part * (long long)(kDv * kH) + h;
+      for (int j = half * 8; j < half * 8 + 8; j += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(trow + j * 32, v[0]);
+        tmem_ld32(trow + (j + 1) * 32, v[1]);
         tmem_ld_wait();
-        float4 *o4 = reinterpret_cast<float4 *>(orow + j * 32);
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-          o4[x] = make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
-                              __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ob[((j + u) * 32 + x) * kH] = __uint_as_float(v[u][x]);
       }
-      p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
-    } else {
+      if (half == 0) p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
+    } else if (half == 0) {
       p.ml_part[part * kH + h] = make_float2(-INFINITY, 0.f);
     }
   }
@@ -297,43 +325,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the splits of each (row, head): out = sum_c e^{m_c - M} O_c / sum_c e^{m_c - M} l_c.
+// Merge the splits of each (row, head) for 8 output values per CTA:
+// out = sum_c e^{m_c - M} O_c / sum_c e^{m_c - M} l_c, one thread per head.
+constexpr int kCombVals = 8;
+constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(128)
     attn_combine_kernel(const float *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-  const int t = blockIdx.x, h = blockIdx.y;
-  __shared__ float wsh[64];
-  __shared__ float s_inv, s_lse;
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int c = 0; c < splits; ++c) M = fmaxf(M, ml_part[((long long)t * splits + c) * kH + h].x);
-    float Lsum = 0.f;
-    for (int c = 0; c < splits; ++c) {
-      const float2 ml = ml_part[((long long)t * splits + c) * kH + h];
-      const float wgt = (M == -INFINITY || ml.y == 0.f) ? 0.f : __expf(ml.x - M);
-      wsh[c] = wgt;
-      Lsum += wgt * ml.y;
-    }
-    s_inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    s_lse = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
-  }
-  __syncthreads();
-  const int d = threadIdx.x * 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int t = blockIdx.x, d0 = blockIdx.y * kCombVals, h = threadIdx.x;
+  const float2 *ml = ml_part + (long long)t * splits * kH + h;
+  float M = -INFINITY;
   for (int c = 0; c < splits; ++c) {
-    const float wgt = wsh[c];
-    if (wgt == 0.f) continue;
-    const float4 o = __ldcs(reinterpret_cast<const float4 *>(o_part + (((long long)t * splits + c) * kH + h) * kDv + d));
-    acc.x = fmaf(wgt, o.x, acc.x);
-    acc.y = fmaf(wgt, o.y, acc.y);
-    acc.z = fmaf(wgt, o.z, acc.z);
-    acc.w = fmaf(wgt, o.w, acc.w);
+    const float2 v = ml[c * kH];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
   }
-  const float inv = s_inv;
-  __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(out + ((long long)t * kH + h) * kDv + d);
-  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  if (lse && threadIdx.x == 0) lse[(long long)t * kH + h] = s_lse;
+  float acc[kCombVals];
+#pragma unroll
+  for (int x = 0; x < kCombVals; ++x) acc[x] = 0.f;
+  float Lsum = 0.f;
+  const float *ob = o_part + (long long)t * splits * (kDv * kH) + (long long)d0 * kH + h;
+  for (int c0 = 0; c0 < splits; c0 += 4) {
+    float vals[4][kCombVals], wgt[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // all loads of four splits in flight together
+      const int c = c0 + u;
+      const float2 v = c < splits ? ml[c * kH] : make_float2(-INFINITY, 0.f);
+      wgt[u] = v.y > 0.f ? __expf(v.x - M) : 0.f;
+      Lsum = fmaf(wgt[u], v.y > 0.f ? v.y : 0.f, Lsum);
+#pragma unroll
+      for (int x = 0; x < kCombVals; ++x)
+        vals[u][x] = wgt[u] != 0.f ? __ldcs(ob + (long long)c * (kDv * kH) + x * kH) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int x = 0; x < kCombVals; ++x) acc[x] = fmaf(wgt[u], vals[u][x], acc[x]);
+  }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  *reinterpret_cast<uint4 *>(out + ((long long)t * kH + h) * kDv + d0) =
+      make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                 pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+  if (lse && blockIdx.y == 0) lse[(long long)t * kH + h] = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
 }
 
 // ------------------------------------------------------------------ host
@@ -417,7 +449,7 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     attn_bf16_kernel<<<nr * pl.splits, kThreads, kSmem, stream>>>(tq, p);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    attn_combine_kernel<<<dim3(nr, kH), 128, 0, stream>>>(
+    attn_combine_kernel<<<dim3(nr, kDv / kCombVals), 128, 0, stream>>>(
         p.o_part, p.ml_part, pl.splits, static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
         lse ? lse + (size_t)r0 * kH : nullptr);
     err = cudaGetLastError();
@@ -496,7 +528,7 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   attn_bf16_kernel<<<T * pl.splits, kThreads, kSmem, stream>>>(tq, p);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  attn_combine_kernel<<<dim3(T, kH), 128, 0, stream>>>(p.o_part, p.ml_part, pl.splits,
+  attn_combine_kernel<<<dim3(T, kDv / kCombVals), 128, 0, stream>>>(p.o_part, p.ml_part, pl.splits,
                                                         static_cast<__nv_bfloat16 *>(out), lse);
   return cudaGetLastError();
 }
