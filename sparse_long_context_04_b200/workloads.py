@@ -119,7 +119,10 @@ def _rng(seed: int, *names) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence(key)))
 
 
-def _normal(seed, name, shape, chunk_rows=4096, threads=None) -> np.ndarray:
+_CHUNK_ROWS = 4096
+
+
+def _normal(seed, name, shape, chunk_rows=_CHUNK_ROWS, threads=None) -> np.ndarray:
     """N(0,1) float32 array of `shape`, generated in row chunks from independent streams."""
     shape = tuple(int(x) for x in shape)
     out = np.empty(shape, dtype=np.float32)
@@ -205,7 +208,9 @@ def make_inputs(spec: Spec) -> Inputs:
     # ---- query side (iid) ----
     qI = _normal(seed, "q_idx", (T, spec.H_I, spec.d_I))
     w = _normal(seed, "w", (T, spec.H_I)) * np.float32(spec.w_std)
-    q = _normal(seed, "q", (T, spec.H, spec.Dk))
+    big_q = spec.plant != "frac" and T * spec.H * spec.Dk > (1 << 28)
+    # large prefill queries are generated and encoded chunk by chunk (same values)
+    q = None if big_q else _normal(seed, "q", (T, spec.H, spec.Dk))
 
     # ---- key side, per sequence in logical order ----
     kI_seq, kv_seq = [], []
@@ -243,7 +248,14 @@ def make_inputs(spec: Spec) -> Inputs:
     # ---- encode ----
     if spec.fp8:
         q_idx, q_scale = encode_e4m3_per_token(qI)
-        q_t = encode_bf16(q)
+        if big_q:
+            q_t = torch.empty((T, spec.H, spec.Dk), dtype=torch.bfloat16)
+            for r0 in range(0, T, _CHUNK_ROWS):
+                r1 = min(T, r0 + _CHUNK_ROWS)
+                g = _rng(seed, "q", r0)
+                q_t[r0:r1] = encode_bf16(g.standard_normal((r1 - r0, spec.H, spec.Dk), dtype=np.float32))
+        else:
+            q_t = encode_bf16(q)
     else:
         q_idx, q_scale = torch.from_numpy(qI), None
         q_t = torch.from_numpy(q)
