@@ -142,7 +142,7 @@ dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt,
  * device memory up front, or a serving loop where cudaMalloc's implicit device
  * synchronisation is not allowed. Every GPU that loads the library holds the
  * 40 MiB until the process exits.
- *   - A call needs T * ceil(k/256) * 263168 bytes of scratch (16 decode rows at
+ *   - A call needs T * ceil(k/256) * 132096 bytes of scratch (39 decode rows at
  *     k = 2048 fit); larger calls return DSA_ERR_TOO_LARGE and launch nothing.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any

@@ -18,6 +18,7 @@
 //      second kernel merges the splits of each row with log-sum-exp weights.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <mutex>
 #include <math.h>
 
@@ -56,7 +57,8 @@ struct Params {
   int keys_per_split;
   float scale_log2;   // softmax_scale * log2(e)
   float scale;
-  float *o_part;      // [rows][splits][512 values][128 heads] (head-minor: coalesced stores)
+  __half *o_part;     // [rows][splits][512 values][128 heads] (head-minor: coalesced stores),
+                      // each split's output normalised by its own softmax sum
   float2 *ml_part;    // [rows][splits][128]: (max * scale, sum)
   Layout L;
   ErrCtx e;
@@ -246,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[2][32];
         tmem_ld32(trow + j * 32, v[0]);
         if (j + 1 < j1) tmem_ld32(trow + (j + 1) * 32, v[1]);
-        tmem_ld_wait();
+        tmem_ld_wait(v[0]);
+        tmem_ld_wait(v[1]);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           if (j + u >= j1) break;
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = j0; j < j1; ++j) {
         uint32_t v[32];
         tmem_ld32(trow + j * 32, v);
-        tmem_ld_wait();
+        tmem_ld_wait(v);
         const uint32_t vm = s_valid[j];
         uint32_t pk[16];
 #pragma unroll
@@ -297,17 +300,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = mbar_wait(o_full, 0, p.e, 0x531);
     if (ok) {
       tc_fence_after();
-      // this warp's 256 output columns; stores are head-minor so each warp writes whole lines
-      float *ob = p.o_part + part * (long long)(kDv * kH) + h;
+      // this warp's 256 output columns, normalised by the split's own sum: a convex
+      // combination of value rows, so fp16 keeps ~1e-3 absolute accuracy. Stores are
+      // head-minor so that each warp writes whole lines.
+      __half *ob = p.o_part + part * (long long)(kDv * kH) + h;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
       for (int j = half * 8; j < half * 8 + 8; j += 2) {
         uint32_t v[2][32];
         tmem_ld32(trow + j * 32, v[0]);
         tmem_ld32(trow + (j + 1) * 32, v[1]);
-        tmem_ld_wait();
+        tmem_ld_wait(v[0]);
+        tmem_ld_wait(v[1]);
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
-          for (int x = 0; x < 32; ++x) ob[((j + u) * 32 + x) * kH] = __uint_as_float(v[u][x]);
+          for (int x = 0; x < 32; ++x) ob[((j + u) * 32 + x) * kH] = __float2half_rn(__uint_as_float(v[u][x]) * inv_l);
       }
       if (half == 0) p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
     } else if (half == 0) {
@@ -325,12 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the splits of each (row, head) for 8 output values per CTA:
-// out = sum_c e^{m_c - M} O_c / sum_c e^{m_c - M} l_c, one thread per head.
+// Merge the splits of each (row, head) for 8 output values per CTA, one thread per
+// head. With O_c the split's output already divided by its sum l_c:
+// out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c.
 constexpr int kCombVals = 8;
 constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(128)
-    attn_combine_kernel(const float *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
+    attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   const int t = blockIdx.x, d0 = blockIdx.y * kCombVals, h = threadIdx.x;
   const float2 *ml = ml_part + (long long)t * splits * kH + h;
@@ -343,18 +351,18 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int x = 0; x < kCombVals; ++x) acc[x] = 0.f;
   float Lsum = 0.f;
-  const float *ob = o_part + (long long)t * splits * (kDv * kH) + (long long)d0 * kH + h;
+  const __half *ob = o_part + (long long)t * splits * (kDv * kH) + (long long)d0 * kH + h;
   for (int c0 = 0; c0 < splits; c0 += 4) {
     float vals[4][kCombVals], wgt[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {  // all loads of four splits in flight together
       const int c = c0 + u;
       const float2 v = c < splits ? ml[c * kH] : make_float2(-INFINITY, 0.f);
-      wgt[u] = v.y > 0.f ? __expf(v.x - M) : 0.f;
-      Lsum = fmaf(wgt[u], v.y > 0.f ? v.y : 0.f, Lsum);
+      wgt[u] = v.y > 0.f ? __expf(v.x - M) * v.y : 0.f;  // the split's share before normalising
+      Lsum += wgt[u];
 #pragma unroll
       for (int x = 0; x < kCombVals; ++x)
-        vals[u][x] = wgt[u] != 0.f ? __ldcs(ob + (long long)c * (kDv * kH) + x * kH) : 0.f;
+        vals[u][x] = wgt[u] != 0.f ? __half2float(__ldcs(ob + (long long)c * (kDv * kH) + x * kH)) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u)
@@ -399,7 +407,7 @@ bool make_q_map(CUtensorMap *m, const void *q, unsigned long long rows) {
 }
 
 size_t part_bytes_per_row(int splits) {
-  return (size_t)splits * kH * (kDv * sizeof(float) + sizeof(float2));
+  return (size_t)splits * kH * (kDv * sizeof(__half) + sizeof(float2));
 }
 
 }  // namespace
@@ -434,9 +442,9 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
   p.keys_per_split = pl.keys_per_split;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.o_part = static_cast<float *>(ws);
+  p.o_part = static_cast<__half *>(ws);
   p.ml_part = reinterpret_cast<float2 *>(static_cast<char *>(ws) +
-                                         (size_t)rows_max * pl.splits * kH * kDv * sizeof(float));
+                                         (size_t)rows_max * pl.splits * kH * kDv * sizeof(__half));
   p.e = e;
   for (int r0 = 0; r0 < T; r0 += kRowsPerLaunch) {
     const int nr = T - r0 < kRowsPerLaunch ? T - r0 : kRowsPerLaunch;
@@ -520,9 +528,9 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   p.keys_per_split = pl.keys_per_split;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.o_part = static_cast<float *>(scratch);
+  p.o_part = static_cast<__half *>(scratch);
   p.ml_part = reinterpret_cast<float2 *>(static_cast<char *>(scratch) +
-                                         (size_t)T * pl.splits * kH * kDv * sizeof(float));
+                                         (size_t)T * pl.splits * kH * kDv * sizeof(__half));
   p.L = L;
   p.e = e;
   attn_bf16_kernel<<<T * pl.splits, kThreads, kSmem, stream>>>(tq, p);

@@ -547,29 +547,39 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(a_empty + st);  // keys and scales of this stage are no longer read here
           const int nrows = cur.rows();
+          // this warp's accumulator columns: kTokPerWarp tokens x 64 heads, read as
+          // 32-column chunks with the next chunk's TMEM load in flight during the math
+          constexpr int kCh = kTokPerWarp * 2;
+          const int gi0 = G == 1 ? 0 : grp * 2;
+          const uint32_t tb = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + gi0 * kHI);
+          uint32_t va[32], vb[32];
+          tmem_ld32(tb, va);
+          tmem_ld_wait(va);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four independent chains
 #pragma unroll
-          for (int tt = 0; tt < kTokPerWarp; ++tt) {
-            const int gi = G == 1 ? 0 : grp * 2 + tt;
-            uint32_t v[2][32];
-            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + gi * kHI);
-            tmem_ld32(taddr, v[0]);
-            tmem_ld32(taddr + 32, v[1]);
-            const float4 *w4 = reinterpret_cast<const float4 *>(sW + (slot * G + gi) * kHI);
-            tmem_ld_wait();
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four independent chains
+          for (int c = 0; c < kCh; ++c) {
+            uint32_t(&cv)[32] = (c & 1) ? vb : va;
+            uint32_t(&nv)[32] = (c & 1) ? va : vb;
+            if (c + 1 < kCh) tmem_ld32(tb + (uint32_t)((c + 1) * 32), nv);
+            const int tt = c >> 1;
+            const float4 *w4 = reinterpret_cast<const float4 *>(sW + (slot * G + gi0 + tt) * kHI + (c & 1) * 32);
 #pragma unroll
-            for (int j4 = 0; j4 < kHI / 4; ++j4) {
+            for (int j4 = 0; j4 < 8; ++j4) {
               const float4 wv = w4[j4];
-              const uint32_t *vv = v[j4 >> 3] + (j4 & 7) * 4;
-              a0 = fmaf(wv.x, fmaxf(__uint_as_float(vv[0]), 0.f), a0);
-              a1 = fmaf(wv.y, fmaxf(__uint_as_float(vv[1]), 0.f), a1);
-              a2 = fmaf(wv.z, fmaxf(__uint_as_float(vv[2]), 0.f), a2);
-              a3 = fmaf(wv.w, fmaxf(__uint_as_float(vv[3]), 0.f), a3);
+              a0 = fmaf(wv.x, fmaxf(__uint_as_float(cv[4 * j4]), 0.f), a0);
+              a1 = fmaf(wv.y, fmaxf(__uint_as_float(cv[4 * j4 + 1]), 0.f), a1);
+              a2 = fmaf(wv.z, fmaxf(__uint_as_float(cv[4 * j4 + 2]), 0.f), a2);
+              a3 = fmaf(wv.w, fmaxf(__uint_as_float(cv[4 * j4 + 3]), 0.f), a3);
             }
-            const float acc = (a0 + a1) + (a2 + a3);
-            const long long pos = cur.s.p_first + (long long)cur.i * G + gi;
-            const int t = cur.row0() + gi;
-            if (gi < nrows && key_ok && s <= pos) p.scores[(long long)t * p.ld + s] = acc * qs[tt] * sk;
+            if (c & 1) {  // the token's 64 heads are summed: scale and store
+              const int gi = gi0 + tt;
+              const float acc = (a0 + a1) + (a2 + a3);
+              a0 = a1 = a2 = a3 = 0.f;
+              const long long pos = cur.s.p_first + (long long)cur.i * G + gi;
+              const int t = cur.row0() + gi;
+              if (gi < nrows && key_ok && s <= pos) p.scores[(long long)t * p.ld + s] = acc * qs[tt] * sk;
+            }
+            if (c + 1 < kCh) tmem_ld_wait(nv);
           }
           tc_fence_before();
           __syncwarp();

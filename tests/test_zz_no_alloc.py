@@ -42,13 +42,13 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
     ensure_lib()
-    # 32 decode rows x 8 splits of 2048 selected positions need 64 MiB of partials
-    spec = W.DECODE_32K.replace(batch=32, lens=(64,) * 32)
+    # 48 decode rows x 8 splits of 2048 selected positions need 48 MiB of partials
+    spec = W.DECODE_32K.replace(batch=48, lens=(64,) * 48)
     inp = W.make_inputs(spec)
     dc = G.to_device(inp)
-    idx = torch.full((32, spec.k), -1, dtype=torch.int32, device="cuda")
-    out = torch.zeros((32, spec.H, spec.Dv), dtype=torch.bfloat16, device="cuda")
-    lse = torch.zeros((32, spec.H), dtype=torch.float32, device="cuda")
+    idx = torch.full((48, spec.k), -1, dtype=torch.int32, device="cuda")
+    out = torch.zeros((48, spec.H, spec.Dv), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((48, spec.H), dtype=torch.float32, device="cuda")
     with pytest.raises(D.DSAError) as ex:
         D.dsa_sparse_mqa_attn_noalloc(dc.q, dc.kv, idx, dc.layout, out, lse, spec.softmax_scale)
     assert ex.value.status == D.DSA_ERR_TOO_LARGE
