@@ -160,33 +160,26 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from sparse_long_context_04_b200 import dist as X
+    world, rank, local = X.rank_info()
 
     if args.impl == "reference":
         return run_reference(args, world, rank)
 
-    import datetime
-
-    import torch.distributed as dist
-
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    X.init("nccl", dev)
 
     from sparse_long_context_04_b200 import build as B
     if rank == 0:
         B.build()
-    if world > 1:
-        dist.barrier()
+    X.barrier()
     from sparse_long_context_04_b200 import device as G
     from sparse_long_context_04_b200 import dsa as D
     from sparse_long_context_04_b200 import workloads as W
 
     spec = W.WORKLOADS[WORKLOAD]
-    spec = spec.replace(seed=spec.seed + 1000 * rank)
+    spec = spec.replace(seed=X.rank_seed(spec.seed, rank))
     if args.len_range:
         spec = spec.replace(len_range=tuple(args.len_range))
     inp = W.make_inputs(spec)
@@ -223,8 +216,7 @@ def main():
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
+    X.barrier()
     torch.cuda.synchronize(dev)
     wt0 = time.perf_counter()
     start.record(stream)
@@ -233,14 +225,10 @@ def main():
     end.record(stream)
     torch.cuda.synchronize(dev)
     wt1 = time.perf_counter()
-    if world > 1:
-        dist.barrier()
+    X.barrier()
     ms = start.elapsed_time(end)
     stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = X.max_over_ranks(ms, dev)
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during timing")
 
@@ -266,19 +254,14 @@ def main():
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    X.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = X.max_over_ranks(e0.elapsed_time(e1), dev)
     # ---- prefill FP8 indexer (tensor-bound): the 8K-token causal prefill
     pf = prefill_indexer(args, dev, G, D, W) if not args.no_prefill else None
     sampler.stop_flag.set()
@@ -286,9 +269,7 @@ def main():
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during the end-to-end loop")
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    X.finish()
     if rank != 0:
         return
 
@@ -302,7 +283,7 @@ def main():
     step_gbs = sum(ab.values()) / step_s / 1e9
     res = {
         "metric": METRIC,
-        "value": world * T * args.steps / (ms / 1e3),
+        "value": X.job_rate(world, T, args.steps, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -333,7 +314,7 @@ def main():
                                "algorithmic_bytes": ab["topk"] + ab["attn"]},
         "step_roofline": {"achieved": step_gbs, "frac": step_gbs / hbm, "algorithmic_bytes": sum(ab.values())},
         "fp8_indexer_prefill": pf,
-        "e2e": {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": X.job_rate(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "api": "dsa_forward"},
         "gpu_launches": 4 * args.steps,

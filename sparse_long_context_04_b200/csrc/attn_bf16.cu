@@ -321,6 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.ml_part[part * kH + h] = make_float2(-INFINITY, 0.f);
     }
   }
+  if (error_raised(p.e)) {
+    // a wait gave up somewhere: copies and MMAs issued before that may still be in flight
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < 50000ull) __nanosleep(1000);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -85,13 +85,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
   return ok != 0;
 }
 
-// Slow path of mbar_wait: sleeping waits, each at most 1 ms, until the phase
+// Slow path of mbar_wait: sleeping waits, each at most 1 ms (and at most the
+// limit), until the phase
 // completes, another wait has timed out, or the deadline passes (DEV_TIMEOUT
 // recorded with `site`).
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const ErrCtx &e, unsigned site) {
   const unsigned long long t0 = globaltimer();
+  const uint32_t hint = (uint32_t)(e.limit < 1000000ull ? e.limit : 1000000ull);  // never sleep past the limit
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (error_raised(e)) return false;
     if (globaltimer() - t0 > e.limit) {
       raise_error(e, DEV_TIMEOUT, site);
