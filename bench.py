@@ -191,6 +191,8 @@ def main():
     lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
     wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
     ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
+    # indexer + top-k, then attention: a kernel and a split-merge kernel per chunk of 296 rows
+    launches_per_step = 2 + 2 * ((T + 295) // 296)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -317,7 +319,7 @@ def main():
         "e2e": {"value": X.job_rate(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "api": "dsa_forward"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(wt0, wt1),
     }
     if world == 1 and not args.no_cpu_baseline:

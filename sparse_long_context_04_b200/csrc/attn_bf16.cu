@@ -69,6 +69,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// 2^x by the MUFU approximation (relative error ~2^-22, far below the bf16 rounding of P)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // the eight softmax/output warps only
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -274,8 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const float a = ((vm >> x) & 1u) ? exp2f(fmaf(__uint_as_float(v[x]), p.scale_log2, -mb)) : 0.f;
-          const float b = ((vm >> (x + 1)) & 1u) ? exp2f(fmaf(__uint_as_float(v[x + 1]), p.scale_log2, -mb)) : 0.f;
+          const float2 z = fma2(make_float2(p.scale_log2, p.scale_log2),
+                                make_float2(__uint_as_float(v[x]), __uint_as_float(v[x + 1])), make_float2(-mb, -mb));
+          const float a = ((vm >> x) & 1u) ? ex2_approx(z.x) : 0.f;
+          const float b = ((vm >> (x + 1)) & 1u) ? ex2_approx(z.y) : 0.f;
           const uint32_t w = pack_bf16(a, b);
           pk[x >> 1] = w;
           __nv_bfloat162 bw = *reinterpret_cast<const __nv_bfloat162 *>(&w);

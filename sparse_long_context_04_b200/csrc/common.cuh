@@ -137,6 +137,19 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- packed fp32
+// {a.x, a.y} += {w.x, w.y} * {x.x, x.y} as one packed fp32x2 FMA (round to nearest)
+__device__ __forceinline__ float2 fma2(float2 w, float2 x, float2 a) {
+  unsigned long long wv, xv, av, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(wv) : "f"(w.x), "f"(w.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x.x), "f"(x.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a.x), "f"(a.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(wv), "l"(xv), "l"(av));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+
 // ---------------------------------------------------------------- TMEM
 // Allocation and deallocation are warp-wide (.sync.aligned).
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

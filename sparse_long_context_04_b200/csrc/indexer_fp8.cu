@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           uint32_t va[32], vb[32];
           tmem_ld32(tb, va);
           tmem_ld_wait(va);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four independent chains
+          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);  // two packed chains
 #pragma unroll
           for (int c = 0; c < kCh; ++c) {
             uint32_t(&cv)[32] = (c & 1) ? vb : va;
@@ -566,15 +566,18 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
               const float4 wv = w4[j4];
-              a0 = fmaf(wv.x, fmaxf(__uint_as_float(cv[4 * j4]), 0.f), a0);
-              a1 = fmaf(wv.y, fmaxf(__uint_as_float(cv[4 * j4 + 1]), 0.f), a1);
-              a2 = fmaf(wv.z, fmaxf(__uint_as_float(cv[4 * j4 + 2]), 0.f), a2);
-              a3 = fmaf(wv.w, fmaxf(__uint_as_float(cv[4 * j4 + 3]), 0.f), a3);
+              const float2 r01 = make_float2(fmaxf(__uint_as_float(cv[4 * j4]), 0.f),
+                                             fmaxf(__uint_as_float(cv[4 * j4 + 1]), 0.f));
+              const float2 r23 = make_float2(fmaxf(__uint_as_float(cv[4 * j4 + 2]), 0.f),
+                                             fmaxf(__uint_as_float(cv[4 * j4 + 3]), 0.f));
+              a01 = fma2(make_float2(wv.x, wv.y), r01, a01);
+              a23 = fma2(make_float2(wv.z, wv.w), r23, a23);
             }
             if (c & 1) {  // the token's 64 heads are summed: scale and store
               const int gi = gi0 + tt;
-              const float acc = (a0 + a1) + (a2 + a3);
-              a0 = a1 = a2 = a3 = 0.f;
+              const float acc = (a01.x + a01.y) + (a23.x + a23.y);
+              a01 = make_float2(0.f, 0.f);
+              a23 = make_float2(0.f, 0.f);
               const long long pos = cur.s.p_first + (long long)cur.i * G + gi;
               const int t = cur.row0() + gi;
               if (gi < nrows && key_ok && s <= pos) p.scores[(long long)t * p.ld + s] = acc * qs[tt] * sk;
