@@ -98,3 +98,32 @@ def test_topk_zero_rows_is_a_no_op():
     D.dsa_topk(scores, 4, lay, idx, T=0)
     torch.cuda.synchronize()
     assert idx.cpu().tolist() == [[3, 3, 3, 3]]
+
+
+@pytest.mark.parametrize("lens", [(131072, 100000, 65536, 40000), (20000, 6000, 2500)])
+def test_topk_few_ties_at_the_threshold_bit_exact(lens):
+    """Scores rounded to 1e-3: a handful of keys tie at the k-th best value, so the
+    selection must take the lowest positions among them (ties resolved on the
+    candidate list, not by the full-radix fallback)."""
+    ensure_lib()
+    k = 2048
+    rng = np.random.default_rng(sum(lens))
+    B = len(lens)
+    n_max = max(lens)
+    ld = (n_max + 3) // 4 * 4
+    host = np.round(rng.standard_normal((B, ld)), 3).astype(np.float32)
+    scores = torch.from_numpy(host).cuda()
+    seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    lay = D.Layout(seq, n_max)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    D.dsa_topk(scores, k, lay, idx)
+    assert D.dsa_get_device_error() == D.DSA_OK
+    got = idx.cpu().numpy()
+    partial_ties = 0
+    for b, L in enumerate(lens):
+        row = host[b, :L]
+        want = O.topk_row(row, k)
+        assert np.array_equal(got[b], want), (b, L)
+        kth = np.sort(row)[::-1][k - 1]
+        partial_ties += (row == kth).sum() > k - (row > kth).sum()
+    assert partial_ties >= 2  # the case under test: only some of the tied keys are taken
