@@ -14,6 +14,7 @@ ranks. --impl reference times the CPU oracle on a bounded sample instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -31,6 +32,22 @@ import torch  # noqa: E402
 METRIC = "DSA tokens/s (indexer+top-k+sparse attn) at 128K decode, % of roofline"
 UNIT = "tokens/s"
 WORKLOAD = "paged_decode_b16_ctx96k_128k"
+
+
+def captured_traffic(name="indexer_fp8_traffic.txt"):
+    """DRAM bytes per launch from a committed ncu capture, or None once the
+    kernel's sources differ from the ones that capture measured."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        kv = dict(line.split("=", 1) for line in open(path).read().splitlines()
+                  if line and not line.startswith("#") and "=" in line)
+        h = hashlib.sha256()
+        for f in kv["sources"].split():
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        return int(kv["traffic_bytes_per_launch"]) if h.hexdigest() == kv["sha256"].strip() else None
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -310,7 +327,7 @@ def main():
             "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
             "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured" else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": ab["indexer"],
-            "traffic": None,
+            "traffic": captured_traffic(),
         },
         "topk_attn_roofline": {"achieved": ta_gbs, "frac": ta_gbs / hbm,
                                "algorithmic_bytes": ab["topk"] + ab["attn"]},
