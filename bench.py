@@ -14,6 +14,7 @@ ranks. --impl reference times the CPU oracle on a bounded sample instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -233,51 +234,100 @@ def main():
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Stage events on every 8th step only: an event between two kernels ends the
+    # overlap of one kernel's tail with the next one's launch (programmatic
+    # dependent launch), so the other steps run back to back as a user's would.
+    every = 8
+    probed = list(range(0, args.steps, every))
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(4)] for i in probed}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     X.barrier()
     torch.cuda.synchronize(dev)
     wt0 = time.perf_counter()
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(evs.get(i))
     end.record(stream)
     torch.cuda.synchronize(dev)
     wt1 = time.perf_counter()
     X.barrier()
     ms = start.elapsed_time(end)
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    stage_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in probed) / len(probed) for j in range(3)]
     ms = X.max_over_ranks(ms, dev)
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during timing")
 
-    # ---- end to end through dsa_forward with host buffers
-    fw = G.Forward(dc, keep_idx=False)
-    host_in = {n: getattr(dc, n).cpu().pin_memory() for n in ("q_idx", "q_scale", "w", "q")}
+    # ---- end to end through dsa_forward with host buffers. Two slots of per-step
+    # device inputs and outputs: step i+1's inputs cross PCIe (own stream) while
+    # step i computes, and step i's output returns (another stream) while step
+    # i+1 computes. Every step still copies its inputs in and its result out.
+    def slot_case():
+        lay = dc.layout
+        seq = lay.seq_lens.clone()
+        pt = None if lay.page_table is None else lay.page_table.clone()
+        cu = None if lay.cu_q is None else lay.cu_q.clone()
+        nl = D.Layout(seq, lay.c.n_max, cu, pt, lay.c.page_size, lay.c.num_pages)
+        return dataclasses.replace(dc, q_idx=dc.q_idx.clone(),
+                                   q_scale=None if dc.q_scale is None else dc.q_scale.clone(),
+                                   w=dc.w.clone(), q=dc.q.clone(), layout=nl)
+
+    slots = [slot_case(), slot_case()]
+    fws = [G.Forward(c, keep_idx=False) for c in slots]
+    names = ("q_idx", "q_scale", "w", "q")
+    host_in = {n: getattr(dc, n).cpu().pin_memory() for n in names if getattr(dc, n) is not None}
     host_in["seq_lens"] = dc.layout.seq_lens.cpu().pin_memory()
-    host_in["page_table"] = dc.layout.page_table.cpu().pin_memory()
-    dev_in = {"q_idx": dc.q_idx, "q_scale": dc.q_scale, "w": dc.w, "q": dc.q,
-              "seq_lens": dc.layout.seq_lens, "page_table": dc.layout.page_table}
-    out_h = torch.empty(fw.out.shape, dtype=fw.out.dtype).pin_memory()
-    lse_h = torch.empty(fw.lse.shape, dtype=fw.lse.dtype).pin_memory()
+    if dc.layout.page_table is not None:
+        host_in["page_table"] = dc.layout.page_table.cpu().pin_memory()
+
+    def dev_in(c):
+        d = {n: getattr(c, n) for n in host_in if n in names}
+        d["seq_lens"] = c.layout.seq_lens
+        if "page_table" in host_in:
+            d["page_table"] = c.layout.page_table
+        return d
+
+    slot_in = [dev_in(c) for c in slots]
+    out_h = [torch.empty(f.out.shape, dtype=f.out.dtype).pin_memory() for f in fws]
+    lse_h = [torch.empty(f.lse.shape, dtype=f.lse.dtype).pin_memory() for f in fws]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size() + lse_h[0].numel() * lse_h[0].element_size()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    out_ready, out_free = [ev(), ev()], [ev(), ev()]
+    for e in in_free + out_free:
+        e.record(stream)
 
-    def e2e_step():
-        for n, h in host_in.items():
-            dev_in[n].copy_(h, non_blocking=True)
-        fw(stream)
-        out_h.copy_(fw.out, non_blocking=True)
-        lse_h.copy_(fw.lse, non_blocking=True)
+    def e2e_step(i):
+        j = i & 1
+        with torch.cuda.stream(s_in):            # inputs of step i into slot j
+            s_in.wait_event(in_free[j])
+            for n, h in host_in.items():
+                slot_in[j][n].copy_(h, non_blocking=True)
+            in_ready[j].record(s_in)
+        stream.wait_event(in_ready[j])          # compute step i
+        stream.wait_event(out_free[j])
+        fws[j](stream)
+        in_free[j].record(stream)
+        out_ready[j].record(stream)
+        with torch.cuda.stream(s_out):           # result of step i back to the host
+            s_out.wait_event(out_ready[j])
+            out_h[j].copy_(fws[j].out, non_blocking=True)
+            lse_h[j].copy_(fws[j].lse, non_blocking=True)
+            out_free[j].record(s_out)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for i in range(args.warmup):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     X.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    s_out_done = torch.cuda.Event()
+    s_out_done.record(s_out)
+    stream.wait_event(s_out_done)               # the last result is on the host inside the timed region
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = X.max_over_ranks(e0.elapsed_time(e1), dev)
@@ -321,7 +371,8 @@ def main():
             "parallelism": f"dp{world} (independent sequences per rank)",
             "l2": "inputs larger than L2: the 242 MB paged indexer-key cache is streamed every step",
         },
-        "stages_us": {"indexer": stage_ms[0] * 1e3, "topk": stage_ms[1] * 1e3, "attention": stage_ms[2] * 1e3},
+        "stages_us": {"indexer": stage_ms[0] * 1e3, "topk": stage_ms[1] * 1e3, "attention": stage_ms[2] * 1e3,
+                      "probed_steps": len(probed)},
         "roofline": {
             "bound": "hbm", "kernel": "indexer_fp8_kernel (decode, N=64)",
             "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
@@ -335,7 +386,9 @@ def main():
         "fp8_indexer_prefill": pf,
         "e2e": {"value": X.job_rate(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "api": "dsa_forward"},
+                "api": "dsa_forward",
+                "pipeline": "two slots: step i+1's inputs in and step i's result out on their own "
+                            "streams while step i computes; every step copies both"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(wt0, wt1),
     }

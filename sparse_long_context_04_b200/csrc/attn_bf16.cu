@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_valid[kMaxKeys / 32];  // bit i: selected entry i is a real row
   __shared__ float s_part[2][kH];              // per-half row max, then row sum
 
+  pdl_prologue();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x / p.splits;     // row within this launch
   const int split = blockIdx.x % p.splits;
@@ -354,6 +355,7 @@ constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(128)
     attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  pdl_prologue();
   const int t = blockIdx.x, d0 = blockIdx.y * kCombVals, h = threadIdx.x;
   const float2 *ml = ml_part + (long long)t * splits * kH + h;
   float M = -INFINITY;
@@ -468,13 +470,12 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     p.idx = idx + (size_t)r0 * k;
     p.L = L;
     p.L.row0 = L.row0 + r0;
-    attn_bf16_kernel<<<nr * pl.splits, kThreads, kSmem, stream>>>(tq, p);
-    err = cudaGetLastError();
+    err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
     if (err != cudaSuccess) return err;
-    attn_combine_kernel<<<dim3(nr, kDv / kCombVals), 128, 0, stream>>>(
-        p.o_part, p.ml_part, pl.splits, static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
-        lse ? lse + (size_t)r0 * kH : nullptr);
-    err = cudaGetLastError();
+    err = launch_kernel(attn_combine_kernel, dim3(nr, kDv / kCombVals), dim3(128), 0, stream, 0,
+                        static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
+                        static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
+                        lse ? lse + (size_t)r0 * kH : nullptr);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
@@ -547,12 +548,11 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
                                          (size_t)T * pl.splits * kH * kDv * sizeof(__half));
   p.L = L;
   p.e = e;
-  attn_bf16_kernel<<<T * pl.splits, kThreads, kSmem, stream>>>(tq, p);
-  err = cudaGetLastError();
+  err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
   if (err != cudaSuccess) return err;
-  attn_combine_kernel<<<dim3(T, kDv / kCombVals), 128, 0, stream>>>(p.o_part, p.ml_part, pl.splits,
-                                                        static_cast<__nv_bfloat16 *>(out), lse);
-  return cudaGetLastError();
+  return launch_kernel(attn_combine_kernel, dim3(T, kDv / kCombVals), dim3(128), 0, stream, 0,
+                       static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
+                       static_cast<__nv_bfloat16 *>(out), lse);
 }
 
 }  // namespace dsa

@@ -127,6 +127,18 @@ __device__ __forceinline__ bool wait_turn(const volatile int *c, int target, con
 }
 
 // ---------------------------------------------------------------- proxies / fences
+// Programmatic dependent launch (kernels launched with programmatic stream
+// serialization): the next kernel on the stream may be scheduled once every CTA
+// of this one has called pdl_launch_dependents(); pdl_wait() returns once the
+// previous kernel has completed and its writes are visible. Every kernel here
+// calls both first thing, so completion stays ordered kernel by kernel.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_prologue() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

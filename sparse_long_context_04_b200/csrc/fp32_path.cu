@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(kIdxThreads)
     indexer_f32_kernel(const float *__restrict__ q, const float *__restrict__ kI, const float *__restrict__ w,
                        int H_I, int d_I, Layout L, float *__restrict__ scores, long long ld, ErrCtx e) {
   extern __shared__ float sq[];  // [H_I*d_I] query heads, then [H_I] weights
+  pdl_prologue();
   const int t = blockIdx.y;
   const RowPos rp = row_position(L, t);
   const int s0 = blockIdx.x * kIdxThreads;
@@ -70,6 +71,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   float *z = smf;                                      // [k]
   long long *rows = reinterpret_cast<long long *>(smf + ((k + 1) & ~1));  // [k]
   __shared__ float red[kAttnThreads / 32];
+  pdl_prologue();
   const int t = blockIdx.x, h = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const RowPos rp = row_position(L, t);
@@ -136,8 +138,8 @@ cudaError_t launch_indexer_f32(const float *q, const float *kI, const float *w, 
   cudaError_t err = cudaFuncSetAttribute(indexer_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((L.n_max + kIdxThreads - 1) / kIdxThreads), (unsigned)T);
-  indexer_f32_kernel<<<grid, kIdxThreads, smem, stream>>>(q, kI, w, H_I, d_I, L, scores, ld, e);
-  return cudaGetLastError();
+  return launch_kernel(indexer_f32_kernel, grid, dim3(kIdxThreads), smem, stream, 0, q, kI, w, H_I, d_I, L, scores,
+                       ld, e);
 }
 
 cudaError_t launch_attn_f32(const float *q, const float *kv, int T, int H, int Dk, int Dv, float scale,
@@ -147,8 +149,8 @@ cudaError_t launch_attn_f32(const float *q, const float *kv, int T, int H, int D
   cudaError_t err = cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)T, (unsigned)H);
-  attn_f32_kernel<<<grid, kAttnThreads, smem, stream>>>(q, kv, H, Dk, Dv, scale, idx, k, L, out, lse, e);
-  return cudaGetLastError();
+  return launch_kernel(attn_f32_kernel, grid, dim3(kAttnThreads), smem, stream, 0, q, kv, H, Dk, Dv, scale, idx, k, L,
+                       out, lse, e);
 }
 
 }  // namespace dsa

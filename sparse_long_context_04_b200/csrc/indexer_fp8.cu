@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   __shared__ long long s_fseq;      // flat index of the first item within that sequence
   __shared__ int s_b_turn;          // query-group loads issued so far (they are issued in group order)
 
+  pdl_prologue();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.L.batch;
 
@@ -649,8 +650,7 @@ cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int n
   cudaError_t err =
       cudaFuncSetAttribute(indexer_fp8_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (err != cudaSuccess) return err;
-  indexer_fp8_kernel<G><<<num_sms, C::kThreads, C::kSmem, stream>>>(tq, tk, p);
-  return cudaGetLastError();
+  return launch_kernel(indexer_fp8_kernel<G>, dim3(num_sms), dim3(C::kThreads), C::kSmem, stream, 0, tq, tk, p);
 }
 
 }  // namespace

@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
   Shared &sm = *reinterpret_cast<Shared *>(smem_raw);
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + ((sizeof(Shared) + 15) & ~size_t(15)));
 
+  pdl_prologue();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int t = blockIdx.x / C;
@@ -578,19 +579,8 @@ cudaError_t launch_c(const float *scores, long long ld, int T, int k, const Layo
   err = cudaFuncSetAttribute(topk_kernel<C>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)T * C);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<C>, scores, ld, k, L, cap, idx, e);
+  return launch_kernel(topk_kernel<C>, dim3((unsigned)T * C), dim3(kThreads), smem, stream, (unsigned)C, scores, ld, k, L,
+                       cap, idx, e);
 }
 
 }  // namespace
