@@ -25,6 +25,8 @@ written from the words):
                    tokens), token selection (top-k value entries) and MLA in MQA
                    mode (one value entry shared by many queries).
   [mundobytes-run] mundobytes.com run guide: the serving command uses page size 64.
+  [mundobytes-kernels] same page, open-kernels paragraph: the indexer kernels are
+                   published in a paged version.
 
 Readings taken where the pages are silent (each also listed in the design doc):
   * I[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]), ReLU per head before the
@@ -261,3 +263,75 @@ def indexer_rows(case: dict, rows, keys_cache=None):
         qI, w, _ = query_row(case, t)
         res[t] = indexer_row(qI, w, kI[:pos + 1])
     return res
+
+
+# ---------------------------------------------------------------------------
+# cache write: one new token per query row into the paged caches
+#   [mundobytes-run] pages of 64 tokens; [mundobytes-kernels] mundobytes.com, the
+#   open-kernels paragraph: the indexer kernels come in a paged version;
+#   [jdon-indexer] the indexer keys are stored and scored in FP8.
+# Readings: one fp32 scale per key token, scale = max|x| / 448 in
+# fp32 (1 when the row is all zero); code = the e4m3 value nearest to x / scale
+# (fp32 division), ties to the even code, saturating at +-448, the sign kept
+# for values that round to zero.
+
+E4M3_MAX = 448.0
+
+
+def encode_e4m3_rne(y: np.ndarray) -> np.ndarray:
+    """e4m3 byte of the representable value nearest to each y (ties to the even
+    code), saturating to +-448; NaN -> 0x7F. The non-negative codes 0x00..0x7E
+    are the format's finite magnitudes in increasing order, so rounding is a
+    search in that table."""
+    y = np.asarray(y, dtype=np.float64)
+    mags = E4M3_TABLE[:127]                      # codes 0x00 .. 0x7E, increasing
+    a = np.minimum(np.abs(y), E4M3_MAX)
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, 126)   # first magnitude >= a
+    lo = np.clip(hi - 1, 0, 126)
+    d_lo = a - mags[lo]
+    d_hi = mags[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0) & (hi != lo))
+    code = np.where(take_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.signbit(y), code | 0x80, code).astype(np.uint8)
+    return np.where(np.isnan(y), np.uint8(0x7F), code).astype(np.uint8)
+
+
+def quantize_key_row(x: np.ndarray):
+    """(e4m3 bytes, fp32 scale) of one indexer key row, in the kernel's fp32
+    arithmetic: scale = float32(max|x|) / float32(448); y = float32(x) / scale."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32) if amax > 0 else np.float32(1.0)
+    y = (x32 / scale).astype(np.float32)
+    return encode_e4m3_rne(y), np.float32(scale)
+
+
+def cache_append(case: dict, k_new: np.ndarray, kv_new_bits: np.ndarray, k_pool: np.ndarray,
+                 kv_pool_bits: np.ndarray, k_scale: np.ndarray = None):
+    """Write row t's new indexer key (quantised) and latent row (bf16 bits, copied)
+    at the row's own position pos_t of its sequence. Returns updated copies.
+
+    Paged (page_size 64): k_pool uint8 [pages][8448] = [64 x d_I codes][64 fp32
+    scales]; kv_pool_bits uint16 [pages*64][Dk]. Contiguous: k_pool uint8
+    [B][n_max][d_I], k_scale float32 [B][n_max], kv_pool_bits [B][n_max][Dk]."""
+    k_pool = k_pool.copy()
+    kv_pool_bits = kv_pool_bits.copy()
+    k_scale = None if k_scale is None else k_scale.copy()
+    P = int(case["page_size"])
+    d_I = k_new.shape[1]
+    for t in range(k_new.shape[0]):
+        b = int(case["row_seq"][t])
+        pos = int(case["pos"][t])
+        codes, sc = quantize_key_row(k_new[t])
+        if P:
+            page = int(case["page_table"][b][pos // P])
+            slot = pos % P
+            k_pool[page, slot * d_I:(slot + 1) * d_I] = codes
+            k_pool[page, P * d_I + 4 * slot:P * d_I + 4 * slot + 4] = np.frombuffer(
+                np.float32(sc).tobytes(), dtype=np.uint8)
+            kv_pool_bits[page * P + slot] = kv_new_bits[t]
+        else:
+            k_pool[b, pos] = codes
+            k_scale[b, pos] = sc
+            kv_pool_bits[b, pos] = kv_new_bits[t]
+    return k_pool, kv_pool_bits, k_scale

@@ -343,3 +343,85 @@ def test_paged_addressing_against_hand_built_pool():
     kI, kvr = O.seq_keys(case, 0)
     assert np.array_equal(kI, O.decode_e4m3(kb) * sc[:, None].astype(np.float64))
     assert np.array_equal(kvr, O.decode_bf16(kv))
+
+
+# ---------------------------------------------------------------------------
+# cache write: e4m3 encoding and per-token quantisation (pinned to the format's
+# grid, not to the oracle's own search)
+
+def _brute_e4m3(y: float) -> int:
+    """Nearest finite e4m3 code by exhaustive search over the 254 finite codes of
+    y's sign (saturating), ties to the code with an even mantissa."""
+    a = min(abs(y), 448.0)
+    best, best_d = None, None
+    for c in range(0x7F):                      # non-negative finite codes
+        v = O.e4m3_value(c)
+        d = abs(v - a)
+        if best is None or d < best_d or (d == best_d and c % 2 == 0):
+            best, best_d = c, d
+    return best | (0x80 if np.signbit(y) else 0)
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    for c in list(range(0x7F)) + list(range(0x80, 0xFF)):
+        assert int(O.encode_e4m3_rne(np.array([O.e4m3_value(c)]))[0]) == c, hex(c)
+
+
+def test_e4m3_encode_midpoints_go_to_the_even_code():
+    for c in range(0x7E):
+        lo, hi = O.e4m3_value(c), O.e4m3_value(c + 1)
+        mid = (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert int(O.encode_e4m3_rne(np.array([mid]))[0]) == even, (hex(c), mid)
+        assert int(O.encode_e4m3_rne(np.array([-mid]))[0]) == even | 0x80
+        # a hair off the midpoint picks the nearer neighbour
+        eps = (hi - lo) * 1e-3
+        assert int(O.encode_e4m3_rne(np.array([mid - eps]))[0]) == c
+        assert int(O.encode_e4m3_rne(np.array([mid + eps]))[0]) == c + 1
+
+
+def test_e4m3_encode_matches_exhaustive_search():
+    rng = np.random.default_rng(7)
+    ys = np.concatenate([rng.standard_normal(400) * 60, rng.standard_normal(200) * 0.01,
+                         [0.0, -0.0, 448.0, 449.0, 464.0, 1e6, -1e6, 2.0 ** -9, 2.0 ** -10, -2.0 ** -10]])
+    got = O.encode_e4m3_rne(ys)
+    want = np.array([_brute_e4m3(float(v)) for v in ys], dtype=np.uint8)
+    assert np.array_equal(got, want)
+    assert int(O.encode_e4m3_rne(np.array([np.nan]))[0]) == 0x7F
+
+
+def test_quantize_key_row_scale_and_error_bound():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(128).astype(np.float32) * 3
+    codes, sc = O.quantize_key_row(x)
+    assert sc == np.float32(np.max(np.abs(x)) / np.float32(448.0))
+    i = int(np.argmax(np.abs(x)))
+    assert codes[i] in (0x7E, 0xFE)                       # the largest element maps to +-448
+    back = O.decode_e4m3(codes) * np.float64(sc)
+    big = np.abs(x) >= 2.0 ** -6 * sc                      # normal range: 3 mantissa bits
+    assert np.all(np.abs(back[big] - x[big]) <= np.abs(x[big]) / 16 + 1e-12)
+    z_codes, z_sc = O.quantize_key_row(np.zeros(128, np.float32))
+    assert z_sc == 1.0 and not z_codes.any()
+
+
+def test_cache_append_writes_only_the_rows_own_slot():
+    rng = np.random.default_rng(5)
+    P, d_I, Dk, pages = 64, 128, 576, 6
+    case = {"page_size": P, "row_seq": np.array([0, 1]), "pos": np.array([70, 5]),
+            "page_table": np.array([[4, 1], [3, 0]])}
+    k_pool = rng.integers(0, 256, (pages, P * d_I + 4 * P), dtype=np.uint8)
+    kv_pool = rng.integers(0, 65536, (pages * P, Dk), dtype=np.uint16)
+    k_new = rng.standard_normal((2, d_I)).astype(np.float32)
+    kv_new = rng.integers(0, 65536, (2, Dk), dtype=np.uint16)
+    k2, kv2, _ = O.cache_append(case, k_new, kv_new, k_pool, kv_pool)
+    # row 0: position 70 -> page_table[0][1] = 1, slot 6; row 1: position 5 -> page 3, slot 5
+    c0, s0 = O.quantize_key_row(k_new[0])
+    c1, s1 = O.quantize_key_row(k_new[1])
+    assert np.array_equal(k2[1, 6 * d_I:7 * d_I], c0)
+    assert np.array_equal(k2[3, 5 * d_I:6 * d_I], c1)
+    assert k2[1, P * d_I + 24:P * d_I + 28].view(np.float32)[0] == s0
+    assert k2[3, P * d_I + 20:P * d_I + 24].view(np.float32)[0] == s1
+    assert np.array_equal(kv2[1 * P + 6], kv_new[0]) and np.array_equal(kv2[3 * P + 5], kv_new[1])
+    changed = np.argwhere(k2 != k_pool)
+    assert set(map(tuple, changed[:, :1].tolist())) <= {(1,), (3,)}
+    assert (kv2 != kv_pool).any(axis=1).sum() <= 2
