@@ -331,6 +331,25 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = X.max_over_ranks(e0.elapsed_time(e1), dev)
+    # ---- cache write of the step's new tokens (the other half of a decode loop):
+    # each sequence's newest indexer key quantised into its page, its latent row copied
+    g = torch.Generator(device=dev).manual_seed(1234)
+    k_new = torch.randn((T, s.d_I), generator=g, device=dev, dtype=torch.float32)
+    kv_new = torch.randn((T, s.Dk), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    k_scale = None if s.page_size else dc.k_scale
+    for _ in range(args.warmup):
+        D.dsa_cache_append(k_new, kv_new, dc.layout, dc.k_idx, dc.kv, k_scale)
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 200
+    a0.record(stream)
+    for _ in range(reps):
+        D.dsa_cache_append(k_new, kv_new, dc.layout, dc.k_idx, dc.kv, k_scale)
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    append_us = a0.elapsed_time(a1) / reps * 1e3
+    if D.dsa_get_device_error() != D.DSA_OK:
+        raise RuntimeError("device error during the cache write")
     # ---- prefill FP8 indexer (tensor-bound): the 8K-token causal prefill
     pf = prefill_indexer(args, dev, G, D, W) if not args.no_prefill else None
     sampler.stop_flag.set()
@@ -389,6 +408,9 @@ def main():
                 "api": "dsa_forward",
                 "pipeline": "two slots: step i+1's inputs in and step i's result out on their own "
                             "streams while step i computes; every step copies both"},
+        "cache_append": {"us": append_us, "rows": T, "api": "dsa_cache_append",
+                         "bytes": T * (s.d_I * 4 + s.d_I + 4 + 4 * s.Dk),
+                         "note": "per call, back to back; not part of the metric's step"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(wt0, wt1),
     }

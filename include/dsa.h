@@ -132,6 +132,33 @@ dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt,
                                void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Cache write for the decode loop (and prefill chunks): the new token of each query
+ * row goes into the caches at the row's own position pos_t (decode: seq_lens[b]-1;
+ * prefill: from cu_q), so that the next indexer and attention calls read it.
+ * mundobytes.com "Deepseek-v3-2-exp": serving with 64-token KV pages (deployment
+ * section) and paged indexer kernels (open-kernels paragraph); jdon.com
+ * "DeepSeek-V3.2-Exp": the indexer keys are FP8.
+ *   k_new    device [T][d_I] fp32 (k_dt = DSA_F32, 16-byte aligned) or bf16
+ *            (DSA_BF16, 8-byte aligned); d_I must be 128. Quantised per token:
+ *            scale = max|x| / 448 in fp32 (1 for an all-zero row), code = the e4m3
+ *            value nearest to x / scale (IEEE fp32 division), ties to even,
+ *            saturating at +-448. Inputs are expected finite.
+ *   kv_new   device [T][Dk] bf16 latent rows (16-byte aligned, Dk a multiple of 8,
+ *            at most 4096), or NULL to write only the indexer key
+ *   lay      the layout the other calls use; it already counts the new token
+ *   k_cache  paged (page_size 64): the indexer-key pool, 8448 bytes per page =
+ *            [64 x 128 code bytes][64 fp32 scales], k_scale = NULL;
+ *            contiguous: [B][n_max][128] code bytes with k_scale [B][n_max] fp32
+ *   kv_cache paged: [num_pages*64][Dk] bf16; contiguous: [B][n_max][Dk] bf16
+ * Writes only the bytes of each row's own slot. A page id out of range is a
+ * device check failure (reported by dsa_get_device_error); rows whose position
+ * lies outside the cache are skipped and reported the same way.
+ */
+dsa_status dsa_cache_append(const void *k_new, dsa_dtype k_dt, const void *kv_new,
+                            int T, int d_I, int Dk, const dsa_seq_layout *lay,
+                            void *k_cache, float *k_scale, void *kv_cache, void *stream);
+
+/*
  * Stage 3 without a caller workspace (no counterpart on the pages; this entry
  * point exists for callers, not for the method).
  * Same computation, arguments and dtype as dsa_sparse_mqa_attn with dt = DSA_BF16,

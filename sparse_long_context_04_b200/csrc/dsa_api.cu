@@ -312,6 +312,30 @@ dsa_status dsa_sparse_mqa_attn_noalloc(const void *q, const void *kv, dsa_dtype 
                                                  static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status dsa_cache_append(const void *k_new, dsa_dtype k_dt, const void *kv_new, int T, int d_I, int Dk,
+                            const dsa_seq_layout *lay, void *k_cache, float *k_scale, void *kv_cache, void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  if (!k_new || !k_cache) return DSA_ERR_INVALID_ARG;
+  if (k_dt != DSA_F32 && k_dt != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  if (d_I != 128) return DSA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(k_new) & (k_dt == DSA_F32 ? 15u : 7u)) != 0) return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_cache) & 3u) != 0) return DSA_ERR_INVALID_ARG;
+  if (L.page_size ? k_scale != nullptr : (k_scale == nullptr || (reinterpret_cast<uintptr_t>(k_scale) & 3u)))
+    return DSA_ERR_INVALID_ARG;
+  if (kv_new) {
+    if (!kv_cache || Dk < 8 || Dk > 4096 || (Dk % 8) != 0 || !a16(kv_new) || !a16(kv_cache))
+      return DSA_ERR_INVALID_ARG;
+  }
+  if (T == 0) return DSA_OK;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_cache_append(k_new, k_dt == DSA_BF16, kv_new, T, Dk, L, k_cache, k_scale, kv_cache, e,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_forward_workspace_size(const dsa_forward_args *a) {
   ErrCtx e;
   int sms;

@@ -75,4 +75,8 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
                                      const Layout &L, void *out, float *lse, const ErrCtx &e, int num_sms,
                                      cudaStream_t stream);
 
+// cache write (cache_append.cu): new indexer key (e4m3 + per-token scale) and latent row per query row
+cudaError_t launch_cache_append(const void *k_new, bool k_bf16, const void *kv_new, int T, int Dk, const Layout &L,
+                                void *k_cache, float *k_scale, void *kv_cache, const ErrCtx &e, cudaStream_t stream);
+
 }  // namespace dsa

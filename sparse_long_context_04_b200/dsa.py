@@ -56,7 +56,8 @@ _lib = None
 
 EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size", "dsa_sparse_mqa_attn",
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
-           "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site")
+           "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site",
+           "dsa_cache_append")
 
 
 def lib() -> ctypes.CDLL:
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_mqa_attn_noalloc.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i,
                                                   ctypes.POINTER(SeqLayout), vp, vp, vp]
         L.dsa_sparse_mqa_attn_noalloc.restype = i
+        L.dsa_cache_append.argtypes = [vp, i, vp, i, i, i, ctypes.POINTER(SeqLayout), vp, vp, vp, vp]
+        L.dsa_cache_append.restype = i
         L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(ForwardArgs)]
         L.dsa_forward_workspace_size.restype = sz
         L.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
@@ -167,6 +170,16 @@ def dsa_sparse_mqa_attn(q, kv, idx, layout: Layout, out, lse, softmax_scale, wor
                                   ctypes.byref(layout.c), _p(out), _p(lse), _p(workspace), ws_bytes,
                                   _stream(stream))
     _check(s, "dsa_sparse_mqa_attn")
+
+
+def dsa_cache_append(k_new, kv_new, layout: Layout, k_cache, kv_cache, k_scale=None, stream=None):
+    """Write each query row's new indexer key (quantised to e4m3 with a per-token
+    scale) and latent row at the row's own position (see include/dsa.h)."""
+    T, d_I = (int(x) for x in k_new.shape)
+    Dk = 0 if kv_new is None else int(kv_new.shape[1])
+    s = lib().dsa_cache_append(_p(k_new), _dt(k_new), _p(kv_new), T, d_I, Dk, ctypes.byref(layout.c),
+                               _p(k_cache), _p(k_scale), _p(kv_cache), _stream(stream))
+    _check(s, "dsa_cache_append")
 
 
 def dsa_sparse_mqa_attn_noalloc(q, kv, idx, layout: Layout, out, lse, softmax_scale, stream=None):
