@@ -173,6 +173,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill FP8 indexer measurement")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="time every workload (stages, forward, roofline fractions), one JSON line each")
     ap.add_argument("--len-range", type=int, nargs=2, default=None,
                     help="override the context-length range (profiling on a smaller case)")
     args = ap.parse_args()
@@ -195,6 +197,12 @@ def main():
     from sparse_long_context_04_b200 import device as G
     from sparse_long_context_04_b200 import dsa as D
     from sparse_long_context_04_b200 import workloads as W
+
+    if args.all_configs:
+        if rank == 0:
+            all_configs(dev, G, D, W)
+        X.finish()
+        return
 
     spec = W.WORKLOADS[WORKLOAD]
     spec = spec.replace(seed=X.rank_seed(spec.seed, rank))
@@ -463,6 +471,82 @@ def prefill_indexer(args, dev, G, D, W, reps=20):
     peak = 2 * bf16
     return {"workload": spec.name, "us": ms * 1e3, "pairs": pairs, "tflops": tf, "peak_tflops": peak,
             "frac": tf / peak, "peak_source": src, "kernel": "indexer_fp8_kernel (prefill, N=256)"}
+
+
+def all_configs(dev, G, D, W):
+    """Every workload once: per-stage CUDA-event times (each stage called on its own),
+    the composed dsa_forward, tokens/s and each stage against its roofline (the larger
+    of bytes / measured HBM and flops / the dtype's peak). One JSON line per workload."""
+    hbm, _ = peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        bf16 = 1590.0
+    fp8 = 2 * bf16
+    for spec, reps in ((W.TINY, 20), (W.DECODE_32K, 50), (W.PREFILL_8K, 5), (W.PREFILL_2X32K, 2),
+                       (W.PAGED_DECODE_128K, 50)):
+        inp = W.make_inputs(spec)
+        dc = G.to_device(inp, dev)
+        T, s = dc.T, spec
+        pos = inp.pos.to(torch.int64)
+        n_pairs = int((pos + 1).sum())
+        n_sel = int(torch.clamp(pos + 1, max=s.k).sum())
+        lens = [int(x) for x in inp.seq_lens.tolist()]
+        scores = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
+        idx = torch.empty((T, s.k), dtype=torch.int32, device=dev)
+        out = torch.empty((T, s.H, s.Dv), dtype=dc.q.dtype, device=dev)
+        lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
+        wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
+        ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
+        stages = {
+            "indexer": lambda: D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout,
+                                                    scores),
+            "topk": lambda: D.dsa_topk(scores, s.k, dc.layout, idx),
+            "attention": lambda: D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws),
+        }
+        ms = {}
+        for name, fn in stages.items():
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms[name] = e0.elapsed_time(e1) / reps
+        fw = G.Forward(dc, keep_idx=False)
+        for _ in range(2):
+            fw()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fw()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        fwd_ms = e0.elapsed_time(e1) / reps
+        if D.dsa_get_device_error() != D.DSA_OK:
+            raise RuntimeError(f"device error on {spec.name}")
+        line = {"mode": "all_configs", "workload": spec.name, "query_rows": T, "tokens_per_s": T / (fwd_ms / 1e3),
+                "forward_ms": fwd_ms, "stages_ms": ms, "dtype": "fp32" if not s.fp8 else "e4m3 indexer + bf16 attention"}
+        if s.fp8:
+            kbytes = sum(lens) * (s.d_I + 4) + T * (s.H_I * s.d_I + 4 + 4 * s.H_I)
+            roof = {
+                "indexer": max((kbytes + n_pairs * 4) / hbm / 1e6, 2 * s.H_I * s.d_I * n_pairs / fp8 / 1e9),
+                "topk": (n_pairs * 4 + T * s.k * 4) / hbm / 1e6,
+                "attention": max((n_sel * s.Dk * 2 + T * s.H * (s.Dk + s.Dv) * 2 + T * s.H * 4) / hbm / 1e6,
+                                 2 * s.H * (s.Dk + s.Dv) * n_sel / bf16 / 1e9),
+            }
+            line["roofline_ms"] = roof
+            line["frac"] = {k: roof[k] / ms[k] for k in roof}
+            line["forward_frac"] = sum(roof.values()) / fwd_ms
+            line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": bf16, "fp8_tflops": fp8}
+        print(json.dumps(line), flush=True)
+        del dc, scores, idx, out, lse, ws, fw
+        torch.cuda.empty_cache()
 
 
 def run_reference(args, world, rank):
