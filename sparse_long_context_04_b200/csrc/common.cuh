@@ -139,6 +139,11 @@ __device__ __forceinline__ void pdl_prologue() {
   pdl_launch_dependents();
 }
 
+// Bring a global line toward L2 ahead of its first use (no register result).
+__device__ __forceinline__ void prefetch_l2(const void *ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -318,6 +318,14 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
       s_fseq = f0 - pre[lo];
       s_range[0] = f0;
       s_range[1] = f1 - f0;
+      if (G == 1 && p.L.page_size && p.L.cu_q == nullptr) {
+        // decode: this CTA's items are key tiles s_fseq.. of sequence lo, two page ids each;
+        // start the page-table reads now so that they overlap the set-up below
+        const int *row = p.L.page_table + (long long)lo * p.L.max_pages;
+        const long long e0 = 2 * s_fseq;
+        const long long e1 = min((long long)p.L.max_pages, e0 + 2 * (f1 - f0));
+        for (long long e = e0 & ~31ll; e < e1 && e < e0 + 256; e += 32) prefetch_l2(row + e);
+      }
     }
     __syncthreads();
   }

@@ -441,36 +441,17 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
     __syncthreads();
     unsigned o = gt_before + sm.sel_before;
     for (int w = 0; w < warp; ++w) o += sm.wgt[w] + sm.wsel[w];
-    // ---- emit this warp's segment in ascending position order: each lane 4 keys,
-    // a warp prefix only when some lane selects one
-    for (int i0 = s0; i0 < s1; i0 += 128) {
-      const int i = i0 + 4 * lane;
-      uint4 q = make_uint4(0, 0, 0, 0);
-      if (i < s1) q = keys4[i >> 2];
-      const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
-      unsigned m = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool sel = i + j < s1 && (kk[j] > thr || (kk[j] == thr && (uint32_t)(lo + i + j) <= tcut));
-        m |= (unsigned)sel << j;
+    // ---- emit this warp's segment in ascending position order, 32 keys per ballot
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i = s0 + lane; i - lane < s1; i += 32) {
+      const uint32_t key = i < s1 ? keys[i] : 0u;
+      const bool sel = i < s1 && (key > thr || (key == thr && (uint32_t)(lo + i) <= tcut));
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+      if (sel) {
+        const unsigned at = o + __popc(m & lt);
+        if (at < (unsigned)k) out[at] = (int)(lo + i);
       }
-      if (__any_sync(0xFFFFFFFFu, m != 0)) {
-        const unsigned c = __popc(m);
-        unsigned incl = c;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const unsigned t2 = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += t2;
-        }
-        unsigned at = o + incl - c;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if ((m >> j) & 1u) {
-            if (at < (unsigned)k) out[at] = (int)(lo + i + j);
-            ++at;
-          }
-        o += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
+      o += __popc(m);
     }
     return;
   }
