@@ -28,7 +28,7 @@ written from the words):
   [mundobytes-kernels] same page, open-kernels paragraph: the indexer kernels are
                    published in a paged version.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * I[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]), ReLU per head before the
     weighted sum; the FP8 per-token scales multiply the dequantised vectors.
   * causal set s <= pos_t, inclusive of the query's own position.
@@ -270,7 +270,7 @@ def indexer_rows(case: dict, rows, keys_cache=None):
 #   [mundobytes-run] pages of 64 tokens; [mundobytes-kernels] mundobytes.com, the
 #   open-kernels paragraph: the indexer kernels come in a paged version;
 #   [jdon-indexer] the indexer keys are stored and scored in FP8.
-# Readings (DESIGN.md): one fp32 scale per key token, scale = max|x| / 448 in
+# Readings: one fp32 scale per key token, scale = max|x| / 448 in
 # fp32 (1 when the row is all zero); code = the e4m3 value nearest to x / scale
 # (fp32 division), ties to the even code, saturating at +-448, the sign kept
 # for values that round to zero.

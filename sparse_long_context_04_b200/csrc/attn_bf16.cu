@@ -351,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // head. With O_c the split's output already divided by its sum l_c:
 // out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c.
 constexpr int kCombVals = 8;
-constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(128)
     attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
