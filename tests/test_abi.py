@@ -58,3 +58,55 @@ def test_host_rejects_bad_arguments_without_gpu(lib):
     lay.page_size = 64
     assert lib.dsa_topk(vp(16), 64, 2, 8, ctypes.byref(lay), vp(16), None) == D.DSA_ERR_INVALID_ARG
     assert lib.dsa_set_wait_limit_ns(0) == D.DSA_ERR_INVALID_ARG
+
+
+def _decode_layout(batch=2, page_size=0):
+    return D.SeqLayout(batch=batch, seq_lens=16, cu_q=None, page_size=page_size,
+                       page_table=32 if page_size else None, max_pages=4 if page_size else 0,
+                       num_pages=8 if page_size else 0, n_max=256)
+
+
+def test_cache_append_rejects_bad_arguments_without_gpu(lib):
+    vp = ctypes.c_void_p
+    A = 4096  # a 16-byte-aligned stand-in address; no call below reaches the device
+    paged, contig = _decode_layout(page_size=64), _decode_layout()
+    ok_paged = dict(k_new=vp(A), k_dt=D.DSA_F32, kv_new=vp(A), T=2, d_I=128, Dk=576, k_cache=vp(A),
+                    k_scale=None, kv_cache=vp(A))
+
+    def call(lay, **kw):
+        a = dict(ok_paged, **kw)
+        return lib.dsa_cache_append(a["k_new"], a["k_dt"], a["kv_new"], a["T"], a["d_I"], a["Dk"],
+                                    ctypes.byref(lay), a["k_cache"], a["k_scale"], a["kv_cache"], None)
+
+    assert call(paged, k_new=None) == D.DSA_ERR_INVALID_ARG
+    assert call(paged, k_dt=D.DSA_E4M3) == D.DSA_ERR_UNSUPPORTED
+    assert call(paged, d_I=64) == D.DSA_ERR_UNSUPPORTED
+    assert call(paged, k_new=vp(A + 4)) == D.DSA_ERR_INVALID_ARG          # fp32 rows need 16-byte alignment
+    assert call(paged, k_scale=vp(A)) == D.DSA_ERR_INVALID_ARG           # paged pools keep scales in the pages
+    assert call(contig) == D.DSA_ERR_INVALID_ARG                          # contiguous caches need k_scale
+    assert call(paged, Dk=580) == D.DSA_ERR_INVALID_ARG                   # latent rows in 16-byte pieces
+    assert call(paged, kv_cache=None) == D.DSA_ERR_INVALID_ARG
+    assert call(paged, T=3) == D.DSA_ERR_INVALID_ARG                      # decode: one row per sequence
+    # nothing to do: accepted without touching the device
+    cu = _decode_layout()
+    cu.cu_q = A
+    assert call(cu, T=0, k_scale=vp(A)) == D.DSA_OK
+
+
+def test_attention_rejects_shapes_without_a_kernel_without_gpu(lib):
+    vp = ctypes.c_void_p
+    A = 4096
+    lay = _decode_layout()
+
+    def attn(dt=D.DSA_BF16, H=128, Dk=576, Dv=512, k=2048, q=A):
+        return lib.dsa_sparse_mqa_attn(vp(q), vp(A), dt, 2, H, Dk, Dv, ctypes.c_float(0.1), vp(A), k,
+                                       ctypes.byref(lay), vp(A), vp(A), vp(A), ctypes.c_size_t(1 << 20), None)
+
+    assert attn(H=64) == D.DSA_ERR_UNSUPPORTED
+    assert attn(Dk=512, Dv=512) == D.DSA_ERR_UNSUPPORTED
+    assert attn(k=16385) == D.DSA_ERR_UNSUPPORTED
+    assert attn(q=A + 2) == D.DSA_ERR_INVALID_ARG
+    assert attn(Dv=600) == D.DSA_ERR_INVALID_ARG                          # the value is a prefix of the key row
+    # the built-in-scratch entry point takes bf16 only
+    assert lib.dsa_sparse_mqa_attn_noalloc(vp(A), vp(A), D.DSA_F32, 2, 8, 64, 32, ctypes.c_float(0.1), vp(A), 64,
+                                           ctypes.byref(lay), vp(A), vp(A), None) == D.DSA_ERR_UNSUPPORTED
