@@ -335,3 +335,35 @@ def cache_append(case: dict, k_new: np.ndarray, kv_new_bits: np.ndarray, k_pool:
             k_scale[b, pos] = sc
             kv_pool_bits[b, pos] = kv_new_bits[t]
     return k_pool, kv_pool_bits, k_scale
+
+
+# ---------------------------------------------------------------------------
+# indexer loss (sparse stage)
+#   [jdon-warmup] jdon.com "DeepSeek-V3.2-Exp", warm-up paragraph: the indexer first
+#   copies how the main attention distributes its attention, trained with a KL
+#   divergence loss; [jdon-sparse-train] same page, sparse-training paragraph: the
+#   indexer and the main model are trained together with separated gradients, the
+#   indexer optimising only its own scoring loss.
+# Readings: the target is the main attention's distribution over the selected set,
+# averaged over the heads (each head's softmax sums to 1, so the mean is
+# L1-normalised); the indexer's distribution is the softmax of its scores over the
+# same set; loss = KL(target || indexer); the indexer's gradient is
+# softmax(I) - target, and no gradient reaches the attention inputs.
+
+def indexer_kl_row(q_t: np.ndarray, kv_rows: np.ndarray, scale: float, scores: np.ndarray):
+    """(loss, target p, d loss / d scores) for one query row over its selected rows.
+
+    q_t [H, Dk] and kv_rows [m, Dk] as float64 values, scores [m] the indexer
+    scores of the same m selected positions."""
+    z = scale * (np.asarray(q_t, np.float64) @ np.asarray(kv_rows, np.float64).T)   # [H, m]
+    z = z - z.max(axis=1, keepdims=True)
+    a = np.exp(z)
+    a /= a.sum(axis=1, keepdims=True)            # each head's attention over the selected set
+    p = a.mean(axis=0)                           # target: mean over heads, sums to 1
+    s = np.asarray(scores, np.float64)
+    s = s - s.max()
+    q = np.exp(s)
+    q /= q.sum()
+    nz = p > 0
+    loss = float(np.sum(p[nz] * (np.log(p[nz]) - np.log(q[nz]))))
+    return loss, p, q - p

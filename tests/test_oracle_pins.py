@@ -425,3 +425,64 @@ def test_cache_append_writes_only_the_rows_own_slot():
     changed = np.argwhere(k2 != k_pool)
     assert set(map(tuple, changed[:, :1].tolist())) <= {(1,), (3,)}
     assert (kv2 != kv_pool).any(axis=1).sum() <= 2
+
+
+# ---------------------------------------------------------------------------
+# indexer loss: pinned by the properties KL must have and by finite differences
+
+def _kl_case(seed, H=4, Dk=16, m=9):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((H, Dk)), rng.standard_normal((m, Dk)), rng.standard_normal(m) * 2
+
+
+def test_indexer_kl_target_is_a_distribution_and_loss_is_nonnegative():
+    q, kv, s = _kl_case(1)
+    loss, p, g = O.indexer_kl_row(q, kv, 0.3, s)
+    assert np.isclose(p.sum(), 1.0) and (p > 0).all()
+    assert loss >= 0.0
+    assert np.isclose(g.sum(), 0.0)              # both distributions sum to 1
+
+
+def test_indexer_kl_vanishes_when_scores_are_log_target_plus_a_constant():
+    q, kv, _ = _kl_case(2)
+    _, p, _ = O.indexer_kl_row(q, kv, 0.3, np.zeros(kv.shape[0]))
+    loss, _, g = O.indexer_kl_row(q, kv, 0.3, np.log(p) + 7.5)
+    assert abs(loss) < 1e-12 and np.abs(g).max() < 1e-12
+
+
+def test_indexer_kl_single_head_two_keys_closed_form():
+    # one head, two keys: p = softmax(z), q = softmax(s); KL written out by hand
+    q = np.array([[1.0, 0.0]])
+    kv = np.array([[2.0, 0.0], [0.0, 0.0]])
+    scale = 0.5
+    z = np.array([1.0, 0.0])
+    p = np.exp(z) / np.exp(z).sum()
+    s = np.array([0.2, -0.4])
+    qq = np.exp(s) / np.exp(s).sum()
+    want = p[0] * np.log(p[0] / qq[0]) + p[1] * np.log(p[1] / qq[1])
+    loss, pp, g = O.indexer_kl_row(q, kv, scale, s)
+    assert np.isclose(loss, want) and np.allclose(pp, p) and np.allclose(g, qq - p)
+
+
+def test_indexer_kl_gradient_matches_finite_differences():
+    q, kv, s = _kl_case(3)
+    _, _, g = O.indexer_kl_row(q, kv, 0.3, s)
+    eps = 1e-6
+    for i in range(len(s)):
+        d = np.zeros_like(s)
+        d[i] = eps
+        num = (O.indexer_kl_row(q, kv, 0.3, s + d)[0] - O.indexer_kl_row(q, kv, 0.3, s - d)[0]) / (2 * eps)
+        assert abs(num - g[i]) < 1e-7, (i, num, g[i])
+
+
+def test_indexer_kl_target_is_the_mean_of_the_heads_attention():
+    # heads that attend to disjoint keys: the target splits the mass evenly between them
+    q = np.array([[50.0, 0.0], [0.0, 50.0]])
+    kv = np.array([[1.0, 0.0], [0.0, 1.0]])
+    _, p, _ = O.indexer_kl_row(q, kv, 1.0, np.zeros(2))
+    assert np.allclose(p, [0.5, 0.5], atol=1e-12)
+    # one sharp head, one flat head: the mean of the softmaxes (0.75, 0.25), not the
+    # softmax of the summed logits (1, 0) nor one head's attention
+    q = np.array([[50.0, 0.0], [0.0, 0.0]])
+    _, p, _ = O.indexer_kl_row(q, kv, 1.0, np.zeros(2))
+    assert np.allclose(p, [0.75, 0.25], atol=1e-12)
