@@ -159,6 +159,33 @@ dsa_status dsa_cache_append(const void *k_new, dsa_dtype k_dt, const void *kv_ne
                             void *k_cache, float *k_scale, void *kv_cache, void *stream);
 
 /*
+ * Indexer training signal on the selected set (sparse stage), loss and gradient.
+ * jdon.com "DeepSeek-V3.2-Exp": warm-up paragraph (the indexer is trained to copy the
+ * main attention's distribution through a KL-divergence loss, the target being the
+ * heads' attention summed and normalised) and sparse-training paragraph (the loss
+ * is taken over the selected set; the indexer's gradient is kept apart from the
+ * main model's). For row t with S_t = {idx[t*k+i] >= 0}:
+ *   p_t(s)   = (1/H) sum_h exp(z_h(s) - lse[t,h]),  z_h(s) = softmax_scale * q[t,h,:] . kv[s,:]
+ *   r_t(s)   = exp(scores[t*ld+s]) / sum_{s' in S_t} exp(scores[t*ld+s'])
+ *   loss[t]  = sum_{s in S_t} p_t(s) * (ln p_t(s) - ln r_t(s))
+ *   grad[t*k+i] = r_t(s_i) - p_t(s_i) = d loss[t] / d scores[t*ld+s_i]  (0 for -1 slots)
+ * lse is the attention's log-sum-exp per head over the same S_t, as
+ * dsa_sparse_mqa_attn returns it, so that p_t is the heads' mean attention.
+ *   q, kv, idx, lay   as for dsa_sparse_mqa_attn (bf16, H = 128, Dk = 576;
+ *                     positions in S_t distinct; kv 16-byte aligned)
+ *   lse      device float32 [T][H];  scores device float32 [T][ld], ld >= the cache extent
+ *   loss     device float32 [T] (written: zeroed and accumulated in the call)
+ *   grad     device float32 [T][k], or NULL to skip the gradient
+ * q, idx, lse, scores, loss and grad 4-byte aligned. Index errors are device
+ * check failures as in dsa_sparse_mqa_attn; a row with an empty S_t gets loss 0.
+ */
+dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt,
+                          int T, int H, int Dk, float softmax_scale,
+                          const int *idx, int k, const dsa_seq_layout *lay,
+                          const float *lse, const float *scores, long long ld,
+                          float *loss, float *grad, void *stream);
+
+/*
  * Stage 3 without a caller workspace (no counterpart on the pages; this entry
  * point exists for callers, not for the method).
  * Same computation, arguments and dtype as dsa_sparse_mqa_attn with dt = DSA_BF16,

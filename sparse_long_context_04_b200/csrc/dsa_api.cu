@@ -336,6 +336,28 @@ dsa_status dsa_cache_append(const void *k_new, dsa_dtype k_dt, const void *kv_ne
                                             static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt, int T, int H, int Dk, float softmax_scale,
+                          const int *idx, int k, const dsa_seq_layout *lay, const float *lse, const float *scores,
+                          long long ld, float *loss, float *grad, void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  if (!q || !kv || !idx || !lse || !scores || !loss || k < 1 || H < 1 || Dk < 1) return DSA_ERR_INVALID_ARG;
+  const long long capn = L.page_size ? (long long)L.max_pages * L.page_size : L.n_max;
+  if (ld < capn) return DSA_ERR_INVALID_ARG;
+  if (dt != DSA_BF16 || H != 128 || Dk != 576 || k > 16384) return DSA_ERR_UNSUPPORTED;
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(lse) |
+                       reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(loss) |
+                       reinterpret_cast<uintptr_t>(grad) | reinterpret_cast<uintptr_t>(idx);
+  if ((a4 & 3u) != 0 || !a16(kv)) return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_indexer_kl(q, kv, T, softmax_scale, idx, k, lse, scores, ld, L, loss, grad, e,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_forward_workspace_size(const dsa_forward_args *a) {
   ErrCtx e;
   int sms;

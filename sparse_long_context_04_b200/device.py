@@ -79,6 +79,16 @@ def attention(dc: DeviceCase, idx: torch.Tensor, out=None, lse=None, workspace=N
     return out, lse
 
 
+def indexer_kl(dc: DeviceCase, idx: torch.Tensor, lse: torch.Tensor, scores: torch.Tensor, loss=None, grad=None,
+               want_grad=True):
+    if loss is None:
+        loss = torch.empty(dc.T, dtype=torch.float32, device=dc.q.device)
+    if grad is None and want_grad:
+        grad = torch.empty(tuple(idx.shape), dtype=torch.float32, device=dc.q.device)
+    D.dsa_indexer_kl(dc.q, dc.kv, idx, dc.layout, lse, scores, loss, dc.inp.spec.softmax_scale, grad)
+    return loss, grad
+
+
 class Forward:
     """dsa_forward with its buffers allocated once (reusable across steps)."""
 

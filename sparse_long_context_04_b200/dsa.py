@@ -57,7 +57,7 @@ _lib = None
 EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size", "dsa_sparse_mqa_attn",
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
            "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site",
-           "dsa_cache_append")
+           "dsa_cache_append", "dsa_indexer_kl")
 
 
 def lib() -> ctypes.CDLL:
@@ -79,6 +79,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_mqa_attn_noalloc.restype = i
         L.dsa_cache_append.argtypes = [vp, i, vp, i, i, i, ctypes.POINTER(SeqLayout), vp, vp, vp, vp]
         L.dsa_cache_append.restype = i
+        L.dsa_indexer_kl.argtypes = [vp, vp, i, i, i, i, ctypes.c_float, vp, i, ctypes.POINTER(SeqLayout), vp, vp,
+                                     ll, vp, vp, vp]
+        L.dsa_indexer_kl.restype = i
         L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(ForwardArgs)]
         L.dsa_forward_workspace_size.restype = sz
         L.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
@@ -180,6 +183,17 @@ def dsa_cache_append(k_new, kv_new, layout: Layout, k_cache, kv_cache, k_scale=N
     s = lib().dsa_cache_append(_p(k_new), _dt(k_new), _p(kv_new), T, d_I, Dk, ctypes.byref(layout.c),
                                _p(k_cache), _p(k_scale), _p(kv_cache), _stream(stream))
     _check(s, "dsa_cache_append")
+
+
+def dsa_indexer_kl(q, kv, idx, layout: Layout, lse, scores, loss, softmax_scale, grad=None, stream=None):
+    """Indexer loss on the selected set: KL(heads' mean attention || softmax of the
+    indexer scores) per row into `loss`, and its gradient with respect to the
+    selected scores into `grad` (see include/dsa.h)."""
+    T, H, Dk = (int(x) for x in q.shape)
+    s = lib().dsa_indexer_kl(_p(q), _p(kv), _dt(q), T, H, Dk, float(softmax_scale), _p(idx), int(idx.shape[1]),
+                             ctypes.byref(layout.c), _p(lse), _p(scores), int(scores.stride(0)), _p(loss), _p(grad),
+                             _stream(stream))
+    _check(s, "dsa_indexer_kl")
 
 
 def dsa_sparse_mqa_attn_noalloc(q, kv, idx, layout: Layout, out, lse, softmax_scale, stream=None):

@@ -110,3 +110,23 @@ def test_attention_rejects_shapes_without_a_kernel_without_gpu(lib):
     # the built-in-scratch entry point takes bf16 only
     assert lib.dsa_sparse_mqa_attn_noalloc(vp(A), vp(A), D.DSA_F32, 2, 8, 64, 32, ctypes.c_float(0.1), vp(A), 64,
                                            ctypes.byref(lay), vp(A), vp(A), None) == D.DSA_ERR_UNSUPPORTED
+
+
+def test_indexer_kl_rejects_bad_arguments_without_gpu(lib):
+    vp = ctypes.c_void_p
+    A = 4096
+    lay = _decode_layout()          # contiguous, n_max 256
+
+    def kl(dt=D.DSA_BF16, H=128, Dk=576, k=2048, ld=256, kv=A, loss=A, grad=A, lse=A, T=2):
+        return lib.dsa_indexer_kl(vp(A), vp(kv), dt, T, H, Dk, ctypes.c_float(0.1), vp(A), k, ctypes.byref(lay),
+                                  vp(lse), vp(A), ld, vp(loss), vp(grad), None)
+
+    assert kl(loss=None) == D.DSA_ERR_INVALID_ARG
+    assert kl(lse=None) == D.DSA_ERR_INVALID_ARG
+    assert kl(ld=252) == D.DSA_ERR_INVALID_ARG                            # score rows shorter than the cache
+    assert kl(dt=D.DSA_F32) == D.DSA_ERR_UNSUPPORTED
+    assert kl(H=64) == D.DSA_ERR_UNSUPPORTED
+    assert kl(k=16385) == D.DSA_ERR_UNSUPPORTED
+    assert kl(kv=A + 8) == D.DSA_ERR_INVALID_ARG                          # latent rows in 16-byte pieces
+    assert kl(grad=A + 2) == D.DSA_ERR_INVALID_ARG
+    assert kl(T=3) == D.DSA_ERR_INVALID_ARG                               # decode: one row per sequence
