@@ -427,6 +427,8 @@ size_t part_bytes_per_row(int splits) {
 
 }  // namespace
 
+bool make_q576_map(CUtensorMap *m, const void *q, unsigned long long rows) { return make_q_map(m, q, rows); }
+
 AttnPlan attn_bf16_plan(int T, int k, int num_sms) {
   (void)T;
   (void)num_sms;

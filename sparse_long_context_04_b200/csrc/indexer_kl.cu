@@ -1,4 +1,5 @@
-// Indexer loss on the selected set (sparse stage) and its gradient.
+// Indexer loss on the selected set (sparse stage) and its gradient, on the
+// tcgen05 tensor cores.
 //
 // jdon.com "DeepSeek-V3.2-Exp": warm-up paragraph (the indexer learns to copy how
 // the main attention distributes its attention, through a KL-divergence loss) and
@@ -10,11 +11,19 @@
 // with lse_h the row's attention log-sum-exp per head (as the attention call
 // returns it), so p is the heads' mean attention over S_t.
 //
-// First path on the CUDA cores: one CTA per (row, 32 selected slots). The row's
-// 128 x 576 bf16 query (rows padded to an odd number of words, so that the 32
-// head lanes of a warp hit 32 banks) and the chunk's 32 latent rows sit in shared
-// memory; thread (head, half) accumulates 16 key dot products in fp32.
+// Work unit (one CTA): row t and 256 of its selected slots.
+//   1. D[256 keys, 128 heads] = K_sel[256, 576] . Q_t[128, 576]^T: the selected
+//      latent rows are the M side (two M = 128 tiles, gathered with cp.async into
+//      128-byte swizzled tiles), the query's head block the N side (TMA); nine
+//      64-dim chunks, tcgen05 kind::f16, fp32 accumulators in TMEM. With the keys
+//      on the TMEM lanes, the sum over heads is a sum along one thread's own row.
+//   2. Meanwhile the four producer warps, their copies issued, reduce the row's
+//      log-sum-exp of the indexer scores over the whole selected set.
+//   3. Eight epilogue warps (one key per thread, two per TMEM lane quadrant) form
+//      p, r, the gradient and the loss terms; one atomic add per CTA and row.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <math.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -23,166 +32,256 @@ namespace dsa {
 namespace {
 
 constexpr int kH = 128, kDk = 576;
-constexpr int kKeysPerCta = 32;
-constexpr int kThreads = 256;                     // (head, half of the keys)
-constexpr int kQStride = kDk + 2;                 // bf16 per padded query row: 289 words (odd)
-constexpr int kSmem = kH * kQStride * 2 + kKeysPerCta * kDk * 2 + 16;
+constexpr int kRowBytes = kDk * 2;             // 1152
+constexpr int kKeys = 256;                     // selected slots per CTA
+constexpr int kChunks = kDk / 64;              // 9 dim chunks of 128 bytes
+constexpr int kStages = 3;
+constexpr int kQTile = kH * 128;               // 16 KiB
+constexpr int kKTile = kKeys * 128;            // 32 KiB
+constexpr int kStage = kQTile + kKTile;        // 48 KiB
+constexpr int kRing = kStages * kStage;        // 144 KiB
+constexpr int kProducers = 128;                // warps 0-3
+constexpr int kMmaWarp = 4;
+constexpr int kEpiWarp0 = 5, kEpiWarps = 8;
+constexpr int kThreads = 32 * (4 + 1 + kEpiWarps);
+constexpr int kSmem = 1024 + kRing + kKeys * 8 + kKeys * 4 + 256;
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct KlParams {
-  const __nv_bfloat16 *q;    // [T][128][576]
-  const __nv_bfloat16 *kv;   // rows of 576
+  const __nv_bfloat16 *kv;
   const int *idx;            // [T][k]
   int k;
+  int splits;
   const float *lse;          // [T][128]
   const float *scores;       // [T][ld]
   long long ld;
-  float scale;
+  float scale_log2;          // softmax_scale * log2(e)
   float *loss;               // [T], zeroed by the launcher
   float *grad;               // [T][k] or nullptr
   Layout L;
   ErrCtx e;
 };
 
-__device__ __forceinline__ float block_sum(float v, float *red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float s = 0.f;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) s += red[w];
-  return s;
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+__device__ __forceinline__ void producers_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// producers publish the row's LSE_I; the epilogue warps wait for it
+__device__ __forceinline__ void lse_arrive() { asm volatile("bar.arrive 3, 384;" ::: "memory"); }
+__device__ __forceinline__ void lse_wait() { asm volatile("bar.sync 3, 384;" ::: "memory"); }
 
-__device__ __forceinline__ float block_max(float v, float *red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float s = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) s = fmaxf(s, red[w]);
-  return s;
-}
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_kl_kernel(const __grid_constant__ CUtensorMap tm_q, const KlParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  unsigned char *ring = base;
+  long long *rows = reinterpret_cast<long long *>(base + kRing);
+  int *spos = reinterpret_cast<int *>(rows + kKeys);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(spos + kKeys);
+  uint64_t *full = bars, *empty = bars + kStages, *s_full = bars + 2 * kStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_full + 1);
+  __shared__ int s_nvalid;
+  __shared__ __align__(16) float s_lse2[kH];   // lse_h * log2(e), read as float2
+  __shared__ float s_red[kEpiWarps];
+  __shared__ float s_pred[kProducers / 32];
+  __shared__ float s_lse_i;
 
-__global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlParams p) {
   pdl_prologue();
-  extern __shared__ __align__(16) unsigned char smem[];
-  __nv_bfloat16 *sq = reinterpret_cast<__nv_bfloat16 *>(smem);            // [128][kQStride]
-  __nv_bfloat16 *skv = sq + kH * kQStride;                                 // [32][576]
-  __shared__ float red[kThreads / 32];
-  __shared__ float s_p[kKeysPerCta];          // target p of each slot
-  __shared__ long long s_row[kKeysPerCta];    // physical row of each slot, -1 = padding
-  __shared__ int s_pos[kKeysPerCta];
-  const int t = blockIdx.x, j0 = blockIdx.y * kKeysPerCta, tid = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x / p.splits;
+  const int k0 = (blockIdx.x % p.splits) * kKeys;
+  const int nk = min(kKeys, p.k - k0);
+  const int *irow = p.idx + (long long)t * p.k;
+
+  // ---- this CTA's slots (-1 entries are padding, anywhere in the list)
+  if (threadIdx.x == 0) s_nvalid = 0;
+  __syncthreads();
   const RowPos rp = row_position(p.L, t);
   const bool row_ok = rp.len <= cache_capacity(p.L);
-
-  // ---- this CTA's slots
-  if (tid < kKeysPerCta) {
+  for (int i = threadIdx.x; i < kKeys; i += kThreads) {
     long long r = -1;
-    int s = -1;
-    const int j = j0 + tid;
-    if (j < p.k) {
-      s = __ldg(p.idx + (long long)t * p.k + j);
+    if (i < nk) {
+      const int s = __ldg(irow + k0 + i);
       if (s >= 0 && s <= rp.pos && row_ok) {
         r = key_row(p.L, rp.b, s, p.e, 0x700);
       } else if (s != -1) {
         raise_error(p.e, DEV_BOUNDS, 0x701);
       }
+      spos[i] = r >= 0 ? s : -1;
     }
-    s_row[tid] = r;
-    s_pos[tid] = r >= 0 ? s : -1;
+    rows[i] = r;
+    if (r >= 0) atomicMax(&s_nvalid, i + 1);
   }
-  // ---- the row's log-sum-exp of the indexer scores over its selected set
-  float mx = -INFINITY;
-  for (int j = tid; j < p.k; j += kThreads) {
-    const int s = row_ok ? __ldg(p.idx + (long long)t * p.k + j) : -1;
-    if (s >= 0 && s <= rp.pos) mx = fmaxf(mx, __ldg(p.scores + (long long)t * p.ld + s));
-  }
-  mx = block_max(mx, red);
-  float se = 0.f;
-  for (int j = tid; j < p.k; j += kThreads) {
-    const int s = row_ok ? __ldg(p.idx + (long long)t * p.k + j) : -1;
-    if (s >= 0 && s <= rp.pos) se += __expf(__ldg(p.scores + (long long)t * p.ld + s) - mx);
-  }
-  se = block_sum(se, red);
-  const float lse_i = se > 0.f ? mx + logf(se) : INFINITY;
-
-  // ---- query row and the chunk's latent rows into shared memory
-  {
-    const uint32_t *qg = reinterpret_cast<const uint32_t *>(p.q + (long long)t * kH * kDk);
-    uint32_t *qs = reinterpret_cast<uint32_t *>(sq);
-    for (int i = tid; i < kH * (kDk / 2); i += kThreads) {
-      const int h = i / (kDk / 2), d2 = i % (kDk / 2);
-      qs[h * (kQStride / 2) + d2] = qg[i];
-    }
-    const char *kvb = reinterpret_cast<const char *>(p.kv);
-    for (int i = tid; i < kKeysPerCta * (kDk * 2 / 16); i += kThreads) {
-      const int key = i / (kDk * 2 / 16), c = i % (kDk * 2 / 16);
-      const long long r = s_row[key];
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r >= 0) v = *reinterpret_cast<const uint4 *>(kvb + r * (kDk * 2) + c * 16);
-      reinterpret_cast<uint4 *>(skv + key * kDk)[c] = v;
-    }
-  }
+  if (threadIdx.x < kH) s_lse2[threadIdx.x] = __ldg(p.lse + (long long)t * kH + threadIdx.x) * kLog2e;
   __syncthreads();
+  const int nvalid = s_nvalid;  // entries at or after nvalid are all padding
+  if (nvalid == 0) {
+    if (p.grad != nullptr && threadIdx.x < nk) p.grad[(long long)t * p.k + k0 + threadIdx.x] = 0.f;
+    return;
+  }
+  const int nt = (nvalid + 127) / 128;  // M = 128 key tiles
+  const int n = nt * 128;
 
-  // ---- z for (head h, 16 keys of this half), then exp(z - lse_h)
-  const int h = tid & (kH - 1), half = tid >> 7;
-  float acc[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) acc[u] = 0.f;
-  const __nv_bfloat162 *qh = reinterpret_cast<const __nv_bfloat162 *>(sq + h * kQStride);
-  const __nv_bfloat162 *kk = reinterpret_cast<const __nv_bfloat162 *>(skv + half * 16 * kDk);
-  for (int d2 = 0; d2 < kDk / 2; ++d2) {
-    const float2 qv = __bfloat1622float2(qh[d2]);
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const float2 kv2 = __bfloat1622float2(kk[u * (kDk / 2) + d2]);
-      acc[u] = fmaf(qv.x, kv2.x, fmaf(qv.y, kv2.y, acc[u]));
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, kProducers + 1);
+      mbar_init(empty + s, 1);
     }
+    mbar_init(s_full, 1);
+    fence_mbar_init();
   }
-  const float lse_h = row_ok ? __ldg(p.lse + (long long)t * kH + h) : 0.f;
-  // exp(z - lse_h), summed over the warp's 32 heads, then over the 4 warps of this half
-  for (int u = 0; u < 16; ++u) {
-    const bool live = s_row[half * 16 + u] >= 0;
-    float e = live ? __expf(fmaf(acc[u], p.scale, -lse_h)) : 0.f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xFFFFFFFFu, e, off);
-    acc[u] = e;  // the warp's 32-head sum, in every lane
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
   }
-  __shared__ float s_wsum[kThreads / 32][16];
-  if ((tid & 31) == 0)
-#pragma unroll
-    for (int u = 0; u < 16; ++u) s_wsum[tid >> 5][u] = acc[u];
+  tc_fence_before();
   __syncthreads();
-  if (tid < kKeysPerCta) {
-    const int hf = tid / 16, u = tid % 16;  // slot tid = half hf, key u of that half
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) s += s_wsum[hf * 4 + w][u];
-    s_p[tid] = s / kH;
-  }
-  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const char *kvb = reinterpret_cast<const char *>(p.kv);
 
-  // ---- loss terms and gradient per slot
-  float c = 0.f;
-  if (tid < kKeysPerCta) {
-    const int j = j0 + tid;
-    const float pj = s_p[tid];
-    float g = 0.f;
-    if (s_row[tid] >= 0) {
-      const float lr = __ldg(p.scores + (long long)t * p.ld + s_pos[tid]) - lse_i;  // log r
-      g = __expf(lr) - pj;
+  if (warp < 4) {
+    // ================= producers: Q chunks by TMA, selected rows by cp.async
+    const int tid = threadIdx.x;
+    if (tid == 0) tma_prefetch_desc(&tm_q);
+    bool ok = true;
+    for (int c = 0; c < kChunks && ok; ++c) {
+      const int st = c % kStages;
+      ok = mbar_wait(empty + st, ((c / kStages) & 1) ^ 1, p.e, 0x710);
+      if (!ok) break;
+      unsigned char *sq = ring + st * kStage;
+      const uint32_t sk = smem_u32(sq + kQTile);
+      if (tid == 0) {
+        mbar_expect_tx(full + st, kQTile);
+        tma_load_2d(sq, &tm_q, full + st, c * 64, t * kH);
+      }
+      for (int q = tid; q < n * 8; q += kProducers) {
+        const int i = q >> 3, u = q & 7;
+        const long long r = rows[i];
+        const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + c * 128 + u * 16;
+        cp_async16_zfill(sk + sw128_off(i, u), src, r >= 0);
+      }
+      cp_async_arrive_noinc(full + st);
+    }
+    // ---- LSE_I over the row's whole selected set, while the copies land
+    float mx = -INFINITY;
+    for (int j = tid; j < p.k; j += kProducers) {
+      const int s = __ldg(irow + j);
+      if (s >= 0 && s <= rp.pos) mx = fmaxf(mx, __ldg(p.scores + (long long)t * p.ld + s));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    if (lane == 0) s_pred[warp] = mx;
+    producers_bar();
+    mx = fmaxf(fmaxf(s_pred[0], s_pred[1]), fmaxf(s_pred[2], s_pred[3]));
+    producers_bar();  // all producers have read the maxima
+    float se = 0.f;
+    for (int j = tid; j < p.k; j += kProducers) {
+      const int s = __ldg(irow + j);
+      if (s >= 0 && s <= rp.pos) se += ex2_approx((__ldg(p.scores + (long long)t * p.ld + s) - mx) * kLog2e);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xFFFFFFFFu, se, off);
+    if (lane == 0) s_pred[warp] = se;
+    producers_bar();
+    if (tid == 0) s_lse_i = mx + logf((s_pred[0] + s_pred[1]) + (s_pred[2] + s_pred[3]));
+    lse_arrive();
+    cp_async_wait_all();  // nothing may still land in shared memory after exit
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer: D[keys, heads] += K_sel . Q^T
+    if (lane == 0) {
+      const uint32_t idesc = instr_desc(1, 1, 0, 0, 128, kH);
+      const uint32_t r0 = smem_u32(ring);
+      bool ok = true;
+      for (int c = 0; c < kChunks && ok; ++c) {
+        const int st = c % kStages;
+        ok = mbar_wait(full + st, (c / kStages) & 1, p.e, 0x720);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qa = r0 + st * kStage, ka = qa + kQTile;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bd = smem_desc(qa + ks * 32, 16, 1024, SW_128B);
+          for (int m = 0; m < nt; ++m)
+            umma_f16(tmem + m * kH, smem_desc(ka + m * 16384 + ks * 32, 16, 1024, SW_128B), bd, idesc,
+                     (c | ks) != 0);
+        }
+        umma_commit(empty + st);
+      }
+      umma_commit(s_full);
+    }
+    __syncwarp();
+  } else {
+    // ================= epilogue: one selected slot per thread
+    const int ew = warp - kEpiWarp0;
+    const int quad = warp & 3, tile = ew >> 2;
+    const int i = tile * 128 + quad * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + tile * kH;
+    float acc = 0.f;
+    bool ok = tile < nt;
+    if (ok) ok = mbar_wait(s_full, 0, p.e, 0x730);
+    if (ok) {
+      tc_fence_after();
+      const float2 sc = make_float2(p.scale_log2, p.scale_log2);
+      float2 a2 = make_float2(0.f, 0.f);
+      for (int j = 0; j < kH / 32; j += 2) {  // two TMEM loads per wait
+        uint32_t v[2][32];
+        tmem_ld32(trow + j * 32, v[0]);
+        tmem_ld32(trow + (j + 1) * 32, v[1]);
+        tmem_ld_wait(v[0]);
+        tmem_ld_wait(v[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            const float2 l2 = *reinterpret_cast<const float2 *>(s_lse2 + (j + u) * 32 + x);
+            const float2 z = fma2(sc, make_float2(__uint_as_float(v[u][x]), __uint_as_float(v[u][x + 1])),
+                                  make_float2(-l2.x, -l2.y));
+            a2.x += ex2_approx(z.x);
+            a2.y += ex2_approx(z.y);
+          }
+      }
+      acc = a2.x + a2.y;
+    }
+    const int s = i < nvalid ? spos[i] : -1;
+    const bool live = ok && s >= 0;
+    const float pj = live ? acc * (1.f / kH) : 0.f;
+    lse_wait();
+    float c = 0.f, g = 0.f;
+    if (live) {
+      const float lr = __ldg(p.scores + (long long)t * p.ld + s) - s_lse_i;  // log r
+      g = ex2_approx(lr * kLog2e) - pj;
       if (pj > 0.f) c = pj * (logf(pj) - lr);
     }
-    if (p.grad != nullptr && j < p.k) p.grad[(long long)t * p.k + j] = g;
+    if (p.grad != nullptr && i < nk) p.grad[(long long)t * p.k + k0 + i] = g;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, off);
+    if (lane == 0) s_red[ew] = c;
+    epilogue_bar();
+    if (ew == 0 && lane == 0) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kEpiWarps; ++w) tot += s_red[w];
+      atomicAdd(p.loss + t, tot);
+    }
   }
-  c = block_sum(c, red);
-  if (tid == 0 && row_ok) atomicAdd(p.loss + t, c);
+  if (error_raised(p.e)) {
+    // a wait gave up somewhere: copies and MMAs issued before that may still be in flight
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < 50000ull) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    if (lane == 0) mbar_wait(s_full, 0, p.e, 0x740);
+    __syncwarp();
+    tmem_dealloc(tmem, 256);
+  }
 }
 
 }  // namespace
@@ -194,21 +293,22 @@ cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale,
   if (err != cudaSuccess) return err;
   err = cudaMemsetAsync(loss, 0, sizeof(float) * (size_t)T, stream);
   if (err != cudaSuccess) return err;
+  CUtensorMap tq;
+  if (!make_q576_map(&tq, q, (unsigned long long)T * kH)) return cudaErrorInvalidValue;
   KlParams p;
-  p.q = static_cast<const __nv_bfloat16 *>(q);
   p.kv = static_cast<const __nv_bfloat16 *>(kv);
   p.idx = idx;
   p.k = k;
+  p.splits = (k + kKeys - 1) / kKeys;
   p.lse = lse;
   p.scores = scores;
   p.ld = ld;
-  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
   p.loss = loss;
   p.grad = grad;
   p.L = L;
   p.e = e;
-  return launch_kernel(indexer_kl_kernel, dim3(T, (k + kKeysPerCta - 1) / kKeysPerCta), dim3(kThreads), kSmem, stream,
-                       0, p);
+  return launch_kernel(indexer_kl_kernel, dim3((unsigned)T * p.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
 }
 
 }  // namespace dsa

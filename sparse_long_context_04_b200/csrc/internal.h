@@ -79,6 +79,10 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
 cudaError_t launch_cache_append(const void *k_new, bool k_bf16, const void *kv_new, int T, int Dk, const Layout &L,
                                 void *k_cache, float *k_scale, void *kv_cache, const ErrCtx &e, cudaStream_t stream);
 
+// TMA map of bf16 query rows of 576 values viewed as [rows][576]: boxes of 64 values x
+// 128 rows (one head block), 128-byte swizzle (attn_bf16.cu)
+bool make_q576_map(CUtensorMap *m, const void *q, unsigned long long rows);
+
 // indexer loss on the selected set and its gradient (indexer_kl.cu): bf16, H = 128, Dk = 576
 cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale, const int *idx, int k,
                               const float *lse, const float *scores, long long ld, const Layout &L, float *loss,
