@@ -340,20 +340,25 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = X.max_over_ranks(e0.elapsed_time(e1), dev)
     # ---- indexer loss on the last step's selection (a training-side call, outside
-    # the metric's step): KL(heads' mean attention || softmax of the selected scores)
+    # the metric's step): KL(heads' mean attention || softmax of the selected scores).
+    # Its 40 MB of inputs fit in L2, so L2 is flushed before every timed call.
     kl_loss = torch.empty(T, dtype=torch.float32, device=dev)
     kl_grad = torch.empty((T, s.k), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         D.dsa_indexer_kl(dc.q, dc.kv, idx, dc.layout, lse, scores, kl_loss, s.softmax_scale, kl_grad)
     torch.cuda.synchronize(dev)
-    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kl_reps = 20
-    k0.record(stream)
-    for _ in range(kl_reps):
+    kl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(kl_reps)]
+    for r in range(kl_reps):
+        flush.fill_(r & 0xFF)
+        kl_ev[r][0].record(stream)
         D.dsa_indexer_kl(dc.q, dc.kv, idx, dc.layout, lse, scores, kl_loss, s.softmax_scale, kl_grad)
-    k1.record(stream)
+        kl_ev[r][1].record(stream)
     torch.cuda.synchronize(dev)
-    kl_us = k0.elapsed_time(k1) / kl_reps * 1e3
+    kl_us = sum(a.elapsed_time(b) for a, b in kl_ev) / kl_reps * 1e3
+    kl_valid = int((idx >= 0).sum())
+    del flush
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during the indexer loss")
     # ---- cache write of the step's new tokens (the other half of a decode loop):
@@ -446,7 +451,7 @@ def main():
         "cache_append": {"us": append_us, "rows": T, "api": "dsa_cache_append",
                          "bytes": T * (s.d_I * 4 + s.d_I + 4 + 4 * s.Dk),
                          "note": "per call, 20 calls per CUDA graph replay; not part of the metric's step"},
-        "indexer_kl": indexer_kl_summary(kl_us, T, s),
+        "indexer_kl": indexer_kl_summary(kl_us, T, s, kl_valid, hbm, hbm_src),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(wt0, wt1),
     }
@@ -458,19 +463,20 @@ def main():
     print(json.dumps(res), flush=True)
 
 
-# fp32 FMA issue rate of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1965 MHz
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
-
-
-def indexer_kl_summary(us, T, s):
-    """Per-call time of the indexer loss and its ALU roofline (the first path
-    computes the H x |S_t| scores on the CUDA cores in fp32)."""
-    flops = 2.0 * T * s.k * s.H * s.Dk
-    tf = flops / (us * 1e-6) / 1e12
-    return {"us": us, "rows": T, "k": s.k, "api": "dsa_indexer_kl", "bound": "alu", "flops": flops,
-            "achieved": tf, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_ALU_TFLOPS,
-            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-            "note": "per call, loss and gradient, 20 calls timed back to back; not part of the metric's step"}
+def indexer_kl_summary(us, T, s, valid, hbm, hbm_src):
+    """Per-call time of the indexer loss and its HBM roofline: each call reads the
+    selected latent rows, the query rows, the selection, the per-head log-sum-exp
+    and the selected scores, and writes the gradient and the loss."""
+    algo = (valid * (s.Dk * 2 + 4) + T * (s.H * s.Dk * 2 + s.H * 4 + 4)
+            + 2 * T * s.k * 4)
+    gbs = algo / (us * 1e-6) / 1e9
+    return {"us": us, "rows": T, "k": s.k, "api": "dsa_indexer_kl", "kernel": "indexer_kl_kernel",
+            "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_call": algo, "flops": 2.0 * valid * s.H * s.Dk,
+            "note": "per call (loss and gradient), L2 flushed before each of 20 timed calls; "
+                    "not part of the metric's step"}
 
 
 def prefill_indexer(args, dev, G, D, W, reps=20):

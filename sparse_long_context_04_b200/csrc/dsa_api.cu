@@ -354,7 +354,7 @@ dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt, int T, in
   ErrCtx e;
   int sms;
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
-  return from_cuda(dsa::launch_indexer_kl(q, kv, T, softmax_scale, idx, k, lse, scores, ld, L, loss, grad, e,
+  return from_cuda(dsa::launch_indexer_kl(q, kv, T, softmax_scale, idx, k, lse, scores, ld, L, loss, grad, e, sms,
                                           static_cast<cudaStream_t>(stream)));
 }
 

@@ -11,7 +11,8 @@
 // with lse_h the row's attention log-sum-exp per head (as the attention call
 // returns it), so p is the heads' mean attention over S_t.
 //
-// Work unit (one CTA): row t and 256 of its selected slots.
+// Work unit (one CTA): row t and up to 256 of its selected slots (fewer when the
+// rows alone would leave SMs idle).
 //   1. D[256 keys, 128 heads] = K_sel[256, 576] . Q_t[128, 576]^T: the selected
 //      latent rows are the M side (two M = 128 tiles, gathered with cp.async into
 //      128-byte swizzled tiles), the query's head block the N side (TMA); nine
@@ -45,6 +46,7 @@ constexpr int kMmaWarp = 4;
 constexpr int kEpiWarp0 = 5, kEpiWarps = 8;
 constexpr int kThreads = 32 * (4 + 1 + kEpiWarps);
 constexpr int kSmem = 1024 + kRing + kKeys * 8 + kKeys * 4 + 256;
+constexpr int kSplitKeysMin = 64;   // keys per CTA are not split below this
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct KlParams {
@@ -52,6 +54,7 @@ struct KlParams {
   const int *idx;            // [T][k]
   int k;
   int splits;
+  int keys_per_split;        // <= 256
   const float *lse;          // [T][128]
   const float *scores;       // [T][ld]
   long long ld;
@@ -82,7 +85,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long *rows = reinterpret_cast<long long *>(base + kRing);
   int *spos = reinterpret_cast<int *>(rows + kKeys);
   uint64_t *bars = reinterpret_cast<uint64_t *>(spos + kKeys);
-  uint64_t *full = bars, *empty = bars + kStages, *s_full = bars + 2 * kStages;
+  // per ring stage: query chunk landed (TMA), key rows landed (cp.async), stage free
+  uint64_t *qfull = bars, *kfull = bars + kStages, *empty = bars + 2 * kStages, *s_full = bars + 3 * kStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_full + 1);
   __shared__ int s_nvalid;
   __shared__ __align__(16) float s_lse2[kH];   // lse_h * log2(e), read as float2
@@ -93,12 +97,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_prologue();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x / p.splits;
-  const int k0 = (blockIdx.x % p.splits) * kKeys;
-  const int nk = min(kKeys, p.k - k0);
+  const int k0 = (blockIdx.x % p.splits) * p.keys_per_split;
+  const int nk = min(p.keys_per_split, p.k - k0);
   const int *irow = p.idx + (long long)t * p.k;
 
+  if (threadIdx.x == 0) {
+    s_nvalid = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(qfull + s, 1);
+      mbar_init(kfull + s, kProducers);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(s_full, 1);
+    fence_mbar_init();
+    // the first query chunks do not depend on the selection: start them now
+    tma_prefetch_desc(&tm_q);
+    for (int c = 0; c < kStages; ++c) {
+      mbar_expect_tx(qfull + c, kQTile);
+      tma_load_2d(ring + c * kStage, &tm_q, qfull + c, c * 64, t * kH);
+    }
+  }
   // ---- this CTA's slots (-1 entries are padding, anywhere in the list)
-  if (threadIdx.x == 0) s_nvalid = 0;
   __syncthreads();
   const RowPos rp = row_position(p.L, t);
   const bool row_ok = rp.len <= cache_capacity(p.L);
@@ -121,19 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nvalid = s_nvalid;  // entries at or after nvalid are all padding
   if (nvalid == 0) {
     if (p.grad != nullptr && threadIdx.x < nk) p.grad[(long long)t * p.k + k0 + threadIdx.x] = 0.f;
+    if (threadIdx.x == 0)  // the early query chunks must land before the CTA exits
+      for (int c = 0; c < kStages; ++c) mbar_wait(qfull + c, 0, p.e, 0x702);
     return;
   }
   const int nt = (nvalid + 127) / 128;  // M = 128 key tiles
   const int n = nt * 128;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full + s, kProducers + 1);
-      mbar_init(empty + s, 1);
-    }
-    mbar_init(s_full, 1);
-    fence_mbar_init();
-  }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
@@ -147,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     // ================= producers: Q chunks by TMA, selected rows by cp.async
     const int tid = threadIdx.x;
-    if (tid == 0) tma_prefetch_desc(&tm_q);
     bool ok = true;
     for (int c = 0; c < kChunks && ok; ++c) {
       const int st = c % kStages;
@@ -155,9 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       unsigned char *sq = ring + st * kStage;
       const uint32_t sk = smem_u32(sq + kQTile);
-      if (tid == 0) {
-        mbar_expect_tx(full + st, kQTile);
-        tma_load_2d(sq, &tm_q, full + st, c * 64, t * kH);
+      if (tid == 0 && c >= kStages) {
+        mbar_expect_tx(qfull + st, kQTile);
+        tma_load_2d(sq, &tm_q, qfull + st, c * 64, t * kH);
       }
       for (int q = tid; q < n * 8; q += kProducers) {
         const int i = q >> 3, u = q & 7;
@@ -165,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + c * 128 + u * 16;
         cp_async16_zfill(sk + sw128_off(i, u), src, r >= 0);
       }
-      cp_async_arrive_noinc(full + st);
+      cp_async_arrive_noinc(kfull + st);
     }
     // ---- LSE_I over the row's whole selected set, while the copies land
     float mx = -INFINITY;
@@ -199,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int c = 0; c < kChunks && ok; ++c) {
         const int st = c % kStages;
-        ok = mbar_wait(full + st, (c / kStages) & 1, p.e, 0x720);
+        ok = mbar_wait(qfull + st, (c / kStages) & 1, p.e, 0x720) &&
+             mbar_wait(kfull + st, (c / kStages) & 1, p.e, 0x721);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qa = r0 + st * kStage, ka = qa + kQTile;
@@ -284,22 +297,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+__global__ void zero_f32_kernel(float *x, int n) {
+  pdl_prologue();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = 0.f;
+}
+
 }  // namespace
 
 cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale, const int *idx, int k,
                               const float *lse, const float *scores, long long ld, const Layout &L, float *loss,
-                              float *grad, const ErrCtx &e, cudaStream_t stream) {
+                              float *grad, const ErrCtx &e, int num_sms, cudaStream_t stream) {
   cudaError_t err = cudaFuncSetAttribute(indexer_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (err != cudaSuccess) return err;
-  err = cudaMemsetAsync(loss, 0, sizeof(float) * (size_t)T, stream);
   if (err != cudaSuccess) return err;
   CUtensorMap tq;
   if (!make_q576_map(&tq, q, (unsigned long long)T * kH)) return cudaErrorInvalidValue;
+  // fewest splits of at most 256 keys; more (down to 64 keys each) while the rows
+  // alone would leave SMs idle
+  int splits = (k + kKeys - 1) / kKeys;
+  const int fill = num_sms / T;
+  const int most = (k + kSplitKeysMin - 1) / kSplitKeysMin;
+  if (fill > splits) splits = fill < most ? fill : most;
+  const int kps = (k + splits - 1) / splits;
   KlParams p;
   p.kv = static_cast<const __nv_bfloat16 *>(kv);
   p.idx = idx;
   p.k = k;
-  p.splits = (k + kKeys - 1) / kKeys;
+  p.keys_per_split = kps;
+  p.splits = (k + kps - 1) / kps;
   p.lse = lse;
   p.scores = scores;
   p.ld = ld;
@@ -308,6 +333,8 @@ cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale,
   p.grad = grad;
   p.L = L;
   p.e = e;
+  err = launch_kernel(zero_f32_kernel, dim3((T + 255) / 256), dim3(256), 0, stream, 0, loss, T);
+  if (err != cudaSuccess) return err;
   return launch_kernel(indexer_kl_kernel, dim3((unsigned)T * p.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
 }
 

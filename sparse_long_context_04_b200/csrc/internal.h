@@ -86,6 +86,6 @@ bool make_q576_map(CUtensorMap *m, const void *q, unsigned long long rows);
 // indexer loss on the selected set and its gradient (indexer_kl.cu): bf16, H = 128, Dk = 576
 cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale, const int *idx, int k,
                               const float *lse, const float *scores, long long ld, const Layout &L, float *loss,
-                              float *grad, const ErrCtx &e, cudaStream_t stream);
+                              float *grad, const ErrCtx &e, int num_sms, cudaStream_t stream);
 
 }  // namespace dsa
