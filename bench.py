@@ -475,6 +475,7 @@ def indexer_kl_summary(us, T, s, valid, hbm, hbm_src):
             "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured"
             else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_call": algo, "flops": 2.0 * valid * s.H * s.Dk,
+            "traffic": captured_traffic("indexer_kl_traffic.txt"),
             "note": "per call (loss and gradient), L2 flushed before each of 20 timed calls; "
                     "not part of the metric's step"}
 
