@@ -367,3 +367,57 @@ def indexer_kl_row(q_t: np.ndarray, kv_rows: np.ndarray, scale: float, scores: n
     nz = p > 0
     loss = float(np.sum(p[nz] * (np.log(p[nz]) - np.log(q[nz]))))
     return loss, p, q - p
+
+
+# ---------------------------------------------------------------------------
+# sparse attention backward (sparse training stage)
+#   [jdon-sparse-train] jdon.com "DeepSeek-V3.2-Exp", sparse-training paragraph: the
+#   main model is trained on the sparse pattern (k = 2048 entries per query token),
+#   separately from the indexer's own loss.
+# Readings: the backward of stage 3 with respect to the query heads and the
+# selected latent rows, for an upstream gradient dO of the output; the selection
+# is piecewise constant and carries no gradient; a position selected by several
+# query rows, or twice by one row, receives the sum of its slots' gradients.
+
+def sparse_attn_backward_row(q_t: np.ndarray, kv_rows: np.ndarray, Dv: int, scale: float, dO: np.ndarray):
+    """(dq [H, Dk], dkv [m, Dk]): the gradients of sum(dO * o) for one query token,
+    o = softmax(scale * q_t . kv_rows^T) @ kv_rows[:, :Dv] per head.
+
+    With P the per-head softmax, dP = dO . v^T and D_h = sum_s P_hs dP_hs:
+    dz = P (dP - D), dq = scale dz . kv, and the row gradient is scale dz^T . q
+    (key, all Dk dims) plus P^T . dO (value, first Dv dims)."""
+    q_t = np.asarray(q_t, np.float64)
+    kv_rows = np.asarray(kv_rows, np.float64)
+    dO = np.asarray(dO, np.float64)
+    z = scale * (q_t @ kv_rows.T)                    # [H, m]
+    P = np.exp(z - z.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    v = kv_rows[:, :Dv]
+    dP = dO @ v.T                                    # [H, m]
+    D = np.sum(P * dP, axis=1, keepdims=True)        # [H, 1] = dO . o per head
+    dz = P * (dP - D)
+    dq = scale * (dz @ kv_rows)                      # [H, Dk]
+    dkv = scale * (dz.T @ q_t)                       # [m, Dk]  through the key
+    dkv[:, :Dv] += P.T @ dO                          # through the value
+    return dq, dkv
+
+
+def sparse_attn_backward_seq(q_rows: np.ndarray, kv_seq: np.ndarray, idx: np.ndarray, Dv: int, scale: float,
+                             dO: np.ndarray):
+    """Backward over the query rows of one sequence: q_rows [R, H, Dk], kv_seq
+    [L, Dk] (the sequence's latent rows by position), idx [R, k] (positions, -1 =
+    padding), dO [R, H, Dv]. Returns dq [R, H, Dk] and dkv [L, Dk], the latter
+    summed over every slot that selected each position. A row with no selected
+    position gets dq = 0."""
+    R, H, Dk = q_rows.shape
+    dq = np.zeros((R, H, Dk))
+    dkv = np.zeros((kv_seq.shape[0], Dk))
+    for r in range(R):
+        sel = np.asarray(idx[r])
+        sel = sel[sel >= 0]
+        if sel.size == 0:
+            continue
+        g_q, g_kv = sparse_attn_backward_row(q_rows[r], kv_seq[sel], Dv, scale, dO[r])
+        dq[r] = g_q
+        np.add.at(dkv, sel, g_kv)
+    return dq, dkv

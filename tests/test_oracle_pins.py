@@ -486,3 +486,107 @@ def test_indexer_kl_target_is_the_mean_of_the_heads_attention():
     q = np.array([[50.0, 0.0], [0.0, 0.0]])
     _, p, _ = O.indexer_kl_row(q, kv, 1.0, np.zeros(2))
     assert np.allclose(p, [0.75, 0.25], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# sparse attention backward: pinned by finite differences of the forward, an
+# independent autograd implementation, a one-key closed form and a translation
+# invariance of the key-only dimensions.
+
+def _attn_loss(q, kv, Dv, scale, dO):
+    o, _ = O.sparse_attn_row(q, kv, Dv, scale)
+    return float(np.sum(dO * o))
+
+
+def test_attn_backward_matches_central_differences():
+    rng = np.random.default_rng(41)
+    H, m, Dk, Dv, scale = 3, 4, 7, 5, 0.37
+    q = rng.normal(size=(H, Dk))
+    kv = rng.normal(size=(m, Dk))
+    dO = rng.normal(size=(H, Dv))
+    dq, dkv = O.sparse_attn_backward_row(q, kv, Dv, scale, dO)
+    eps = 1e-6
+    for arr, grad in ((q, dq), (kv, dkv)):
+        num = np.zeros_like(arr)
+        for ix in np.ndindex(arr.shape):
+            a0 = arr[ix]
+            arr[ix] = a0 + eps
+            lp = _attn_loss(q, kv, Dv, scale, dO)
+            arr[ix] = a0 - eps
+            lm = _attn_loss(q, kv, Dv, scale, dO)
+            arr[ix] = a0
+            num[ix] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+
+
+def test_attn_backward_matches_torch_autograd_fp64():
+    rng = np.random.default_rng(42)
+    H, m, Dk, Dv, scale = 8, 20, 40, 32, 1 / np.sqrt(40)
+    q = rng.normal(size=(H, Dk))
+    kv = rng.normal(size=(m, Dk))
+    dO = rng.normal(size=(H, Dv))
+    tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
+    tkv = torch.tensor(kv, dtype=torch.float64, requires_grad=True)
+    o = torch.softmax(scale * tq @ tkv.T, dim=1) @ tkv[:, :Dv]
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    dq, dkv = O.sparse_attn_backward_row(q, kv, Dv, scale, dO)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dkv, tkv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attn_backward_one_key_closed_form():
+    # one selected row: P = 1 and o = v for every head, so nothing reaches the
+    # query or the key; the value receives the heads' summed output gradient
+    rng = np.random.default_rng(43)
+    H, Dk, Dv = 4, 9, 6
+    q, kv, dO = rng.normal(size=(H, Dk)), rng.normal(size=(1, Dk)), rng.normal(size=(H, Dv))
+    dq, dkv = O.sparse_attn_backward_row(q, kv, Dv, 0.5, dO)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-14)
+    np.testing.assert_allclose(dkv[0, :Dv], dO.sum(axis=0), rtol=1e-13)
+    np.testing.assert_allclose(dkv[0, Dv:], 0.0, atol=1e-14)
+
+
+def test_attn_backward_key_only_dims_sum_to_zero():
+    # adding one vector c to the key-only dims (Dv..Dk) of every selected row shifts
+    # each head's scores by a constant and leaves o unchanged: the rows' gradients in
+    # those dims sum to zero
+    rng = np.random.default_rng(44)
+    H, m, Dk, Dv = 5, 11, 12, 8
+    q, kv, dO = rng.normal(size=(H, Dk)), rng.normal(size=(m, Dk)), rng.normal(size=(H, Dv))
+    _, dkv = O.sparse_attn_backward_row(q, kv, Dv, 0.3, dO)
+    np.testing.assert_allclose(dkv[:, Dv:].sum(axis=0), 0.0, atol=1e-12)
+    assert np.abs(dkv[:, Dv:]).max() > 1e-3      # not zero row by row
+
+
+def test_attn_backward_seq_accumulates_duplicates_and_skips_padding():
+    # finite differences through the whole sequence: rows that share positions, a
+    # position selected twice by one row, -1 padding and a row with nothing selected
+    rng = np.random.default_rng(45)
+    R, H, L, Dk, Dv, scale = 3, 2, 6, 5, 3, 0.45
+    q = rng.normal(size=(R, H, Dk))
+    kv = rng.normal(size=(L, Dk))
+    dO = rng.normal(size=(R, H, Dv))
+    idx = np.array([[0, 2, 2, -1], [-1, 1, 2, 5], [-1, -1, -1, -1]])
+
+    def loss():
+        tot = 0.0
+        for r in range(R):
+            sel = idx[r][idx[r] >= 0]
+            if sel.size:
+                tot += _attn_loss(q[r], kv[sel], Dv, scale, dO[r])
+        return tot
+
+    dq, dkv = O.sparse_attn_backward_seq(q, kv, idx, Dv, scale, dO)
+    eps = 1e-6
+    for arr, grad in ((q, dq), (kv, dkv)):
+        num = np.zeros_like(arr)
+        for ix in np.ndindex(arr.shape):
+            a0 = arr[ix]
+            arr[ix] = a0 + eps
+            lp = loss()
+            arr[ix] = a0 - eps
+            lm = loss()
+            arr[ix] = a0
+            num[ix] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+    assert np.all(dq[2] == 0) and np.all(dkv[[3, 4]] == 0)
