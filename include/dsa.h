@@ -187,6 +187,37 @@ dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt,
                           float *loss, float *grad, void *stream);
 
 /*
+ * Backward of stage 3 for the sparse training stage: gradients of the attention
+ * output with respect to the query heads and the selected latent rows.
+ * jdon.com "DeepSeek-V3.2-Exp", sparse-training paragraph (the main model is trained
+ * on the selected entries only). For row t, head h and s in S_t, with the forward's
+ * lse and output o:
+ *   P = exp(z - lse[t,h]),  z = softmax_scale * q[t,h,:] . kv[s,:]
+ *   dP = dout[t,h,:] . kv[s,0:Dv],  D = dout[t,h,:] . out[t,h,:],  dz = P (dP - D)
+ *   dq[t,h,:]  += softmax_scale * sum_s dz kv[s,:]
+ *   dkv[s,:]   += softmax_scale * sum_h dz q[t,h,:];  dkv[s,0:Dv] += sum_h P dout[t,h,:]
+ * The selection carries no gradient. A position selected by several rows (or twice
+ * by one) receives the sum of its slots' contributions.
+ *   q, kv, idx, lay   as for dsa_sparse_mqa_attn (bf16, H = 128, Dk = 576, Dv = 512)
+ *   out, dout  device bf16 [T][H][Dv]: the forward output and its gradient
+ *   lse        device float32 [T][H]: the forward's log-sum-exp
+ *   dq         device float32 [T][H][Dk], accumulated into (+=)
+ *   dkv        device float32 with the row numbering of kv (contiguous [B][n_max][Dk],
+ *              paged [num_pages*page_size][Dk]), accumulated into (+=)
+ *   workspace  device scratch of dsa_sparse_mqa_attn_backward_workspace_size(T) bytes,
+ *              256-byte aligned
+ * Every contribution is an atomic fp32 add, so the last bits of dq and dkv may
+ * differ between runs. q, kv, out, dout, dq and dkv 16-byte aligned.
+ */
+size_t dsa_sparse_mqa_attn_backward_workspace_size(int T);
+dsa_status dsa_sparse_mqa_attn_backward(const void *q, const void *kv, dsa_dtype dt,
+                                        int T, int H, int Dk, int Dv, float softmax_scale,
+                                        const int *idx, int k, const dsa_seq_layout *lay,
+                                        const void *out, const void *dout, const float *lse,
+                                        float *dq, float *dkv,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Stage 3 without a caller workspace (no counterpart on the pages; this entry
  * point exists for callers, not for the method).
  * Same computation, arguments and dtype as dsa_sparse_mqa_attn with dt = DSA_BF16,

@@ -429,6 +429,18 @@ size_t part_bytes_per_row(int splits) {
 
 bool make_q576_map(CUtensorMap *m, const void *q, unsigned long long rows) { return make_q_map(m, q, rows); }
 
+bool make_bf16_rows_map(CUtensorMap *m, const void *base, unsigned long long rows, unsigned width) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)width, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)width * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kH};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 AttnPlan attn_bf16_plan(int T, int k, int num_sms) {
   (void)T;
   (void)num_sms;

@@ -358,6 +358,31 @@ dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt, int T, in
                                           static_cast<cudaStream_t>(stream)));
 }
 
+size_t dsa_sparse_mqa_attn_backward_workspace_size(int T) { return T > 0 ? dsa::attn_bwd_workspace(T) : 0; }
+
+dsa_status dsa_sparse_mqa_attn_backward(const void *q, const void *kv, dsa_dtype dt, int T, int H, int Dk, int Dv,
+                                        float softmax_scale, const int *idx, int k, const dsa_seq_layout *lay,
+                                        const void *out, const void *dout, const float *lse, float *dq, float *dkv,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  if (!q || !kv || !idx || !out || !dout || !lse || !dq || !dkv || k < 1 || H < 1 || Dk < 1 || Dv < 1 || Dv > Dk)
+    return DSA_ERR_INVALID_ARG;
+  if (dt != DSA_BF16 || H != 128 || Dk != 576 || Dv != 512 || k > 16384) return DSA_ERR_UNSUPPORTED;
+  if (!a16(q) || !a16(kv) || !a16(out) || !a16(dout) || !a16(dq) || !a16(dkv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  if (ws_bytes < dsa::attn_bwd_workspace(T) || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return DSA_ERR_WORKSPACE;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_attn_bwd(q, kv, T, softmax_scale, idx, k, L, out, dout, lse, dq, dkv, workspace, e,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_forward_workspace_size(const dsa_forward_args *a) {
   ErrCtx e;
   int sms;

@@ -82,6 +82,15 @@ cudaError_t launch_cache_append(const void *k_new, bool k_bf16, const void *kv_n
 // TMA map of bf16 query rows of 576 values viewed as [rows][576]: boxes of 64 values x
 // 128 rows (one head block), 128-byte swizzle (attn_bf16.cu)
 bool make_q576_map(CUtensorMap *m, const void *q, unsigned long long rows);
+// the same for bf16 rows of `width` values (a multiple of 64, rows 16-byte aligned)
+bool make_bf16_rows_map(CUtensorMap *m, const void *base, unsigned long long rows, unsigned width);
+
+// sparse attention backward (attn_bwd.cu): bf16, H = 128, Dk = 576, Dv = 512;
+// the workspace holds dO . o per (row, head)
+size_t attn_bwd_workspace(int T);
+cudaError_t launch_attn_bwd(const void *q, const void *kv, int T, float scale, const int *idx, int k,
+                            const Layout &L, const void *out, const void *dout, const float *lse, float *dq,
+                            float *dkv, void *ws, const ErrCtx &e, cudaStream_t stream);
 
 // indexer loss on the selected set and its gradient (indexer_kl.cu): bf16, H = 128, Dk = 576
 cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale, const int *idx, int k,

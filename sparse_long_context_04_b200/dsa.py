@@ -57,7 +57,8 @@ _lib = None
 EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size", "dsa_sparse_mqa_attn",
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
            "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site",
-           "dsa_cache_append", "dsa_indexer_kl")
+           "dsa_cache_append", "dsa_indexer_kl", "dsa_sparse_mqa_attn_backward",
+           "dsa_sparse_mqa_attn_backward_workspace_size")
 
 
 def lib() -> ctypes.CDLL:
@@ -82,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_kl.argtypes = [vp, vp, i, i, i, i, ctypes.c_float, vp, i, ctypes.POINTER(SeqLayout), vp, vp,
                                      ll, vp, vp, vp]
         L.dsa_indexer_kl.restype = i
+        L.dsa_sparse_mqa_attn_backward_workspace_size.argtypes = [i]
+        L.dsa_sparse_mqa_attn_backward_workspace_size.restype = sz
+        L.dsa_sparse_mqa_attn_backward.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i,
+                                                   ctypes.POINTER(SeqLayout), vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_sparse_mqa_attn_backward.restype = i
         L.dsa_forward_workspace_size.argtypes = [ctypes.POINTER(ForwardArgs)]
         L.dsa_forward_workspace_size.restype = sz
         L.dsa_forward.argtypes = [ctypes.POINTER(ForwardArgs), vp, sz, vp]
@@ -194,6 +200,23 @@ def dsa_indexer_kl(q, kv, idx, layout: Layout, lse, scores, loss, softmax_scale,
                              ctypes.byref(layout.c), _p(lse), _p(scores), int(scores.stride(0)), _p(loss), _p(grad),
                              _stream(stream))
     _check(s, "dsa_indexer_kl")
+
+
+def dsa_sparse_mqa_attn_backward_workspace_size(T) -> int:
+    return int(lib().dsa_sparse_mqa_attn_backward_workspace_size(int(T)))
+
+
+def dsa_sparse_mqa_attn_backward(q, kv, idx, layout: Layout, out, dout, lse, dq, dkv, softmax_scale, workspace,
+                                 stream=None):
+    """Gradients of the sparse attention output with respect to q and the selected
+    latent rows, accumulated into dq and dkv (fp32; see include/dsa.h)."""
+    T, H, Dk = (int(x) for x in q.shape)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    s = lib().dsa_sparse_mqa_attn_backward(_p(q), _p(kv), _dt(q), T, H, Dk, int(out.shape[2]),
+                                           float(softmax_scale), _p(idx), int(idx.shape[1]), ctypes.byref(layout.c),
+                                           _p(out), _p(dout), _p(lse), _p(dq), _p(dkv), _p(workspace), ws_bytes,
+                                           _stream(stream))
+    _check(s, "dsa_sparse_mqa_attn_backward")
 
 
 def dsa_sparse_mqa_attn_noalloc(q, kv, idx, layout: Layout, out, lse, softmax_scale, stream=None):

@@ -130,3 +130,27 @@ def test_indexer_kl_rejects_bad_arguments_without_gpu(lib):
     assert kl(kv=A + 8) == D.DSA_ERR_INVALID_ARG                          # latent rows in 16-byte pieces
     assert kl(grad=A + 2) == D.DSA_ERR_INVALID_ARG
     assert kl(T=3) == D.DSA_ERR_INVALID_ARG                               # decode: one row per sequence
+
+
+def test_attention_backward_rejects_bad_arguments_without_gpu(lib):
+    vp = ctypes.c_void_p
+    A = 4096
+    lay = _decode_layout()
+
+    def bwd(dt=D.DSA_BF16, H=128, Dk=576, Dv=512, k=2048, dq=A, lse=A, ws=A, ws_bytes=1 << 20, T=2):
+        return lib.dsa_sparse_mqa_attn_backward(vp(A), vp(A), dt, T, H, Dk, Dv, ctypes.c_float(0.1), vp(A), k,
+                                                ctypes.byref(lay), vp(A), vp(A), vp(lse), vp(dq), vp(A), vp(ws),
+                                                ctypes.c_size_t(ws_bytes), None)
+
+    assert bwd(dq=None) == D.DSA_ERR_INVALID_ARG
+    assert bwd(dt=D.DSA_F32) == D.DSA_ERR_UNSUPPORTED
+    assert bwd(H=64) == D.DSA_ERR_UNSUPPORTED
+    assert bwd(k=16385) == D.DSA_ERR_UNSUPPORTED
+    assert bwd(Dv=600) == D.DSA_ERR_INVALID_ARG                           # the value is a prefix of the row
+    assert bwd(dq=A + 4) == D.DSA_ERR_INVALID_ARG                         # fp32 rows added 16 bytes at a time
+    assert bwd(lse=A + 2) == D.DSA_ERR_INVALID_ARG
+    assert bwd(ws=None) == D.DSA_ERR_WORKSPACE
+    assert bwd(ws_bytes=512) == D.DSA_ERR_WORKSPACE                       # two rows need 1 KiB of dO . o
+    assert bwd(ws=A + 128) == D.DSA_ERR_WORKSPACE
+    assert lib.dsa_sparse_mqa_attn_backward_workspace_size(2) == 1024
+    assert lib.dsa_sparse_mqa_attn_backward_workspace_size(0) == 0
