@@ -173,6 +173,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill FP8 indexer measurement")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the sparse-attention backward on the step's selection")
     ap.add_argument("--all-configs", action="store_true",
                     help="time every workload (stages, forward, roofline fractions), one JSON line each")
     ap.add_argument("--len-range", type=int, nargs=2, default=None,
@@ -361,6 +363,31 @@ def main():
     del flush
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during the indexer loss")
+    # ---- sparse-attention backward on the last step's selection and output (a
+    # training-side call, outside the metric's step), L2 flushed before each call
+    bwd = None
+    if args.backward:
+        g = torch.Generator(device=dev).manual_seed(4321)
+        dout = torch.randn((T, s.H, s.Dv), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        dq = torch.zeros((T, s.H, s.Dk), dtype=torch.float32, device=dev)
+        dkv = torch.zeros(tuple(dc.kv.shape), dtype=torch.float32, device=dev)
+        bws = torch.empty(D.dsa_sparse_mqa_attn_backward_workspace_size(T), dtype=torch.uint8, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            D.dsa_sparse_mqa_attn_backward(dc.q, dc.kv, idx, dc.layout, out, dout, lse, dq, dkv, s.softmax_scale, bws)
+        torch.cuda.synchronize(dev)
+        b_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+        for r, (e0b, e1b) in enumerate(b_ev):
+            flush.fill_(r & 0xFF)
+            e0b.record(stream)
+            D.dsa_sparse_mqa_attn_backward(dc.q, dc.kv, idx, dc.layout, out, dout, lse, dq, dkv, s.softmax_scale, bws)
+            e1b.record(stream)
+        torch.cuda.synchronize(dev)
+        bwd_us = sum(a.elapsed_time(b) for a, b in b_ev) / len(b_ev) * 1e3
+        bwd = (bwd_us, int((idx >= 0).sum()))
+        del flush, dkv
+        if D.dsa_get_device_error() != D.DSA_OK:
+            raise RuntimeError("device error during the attention backward")
     # ---- cache write of the step's new tokens (the other half of a decode loop):
     # each sequence's newest indexer key quantised into its page, its latent row copied
     g = torch.Generator(device=dev).manual_seed(1234)
@@ -452,6 +479,7 @@ def main():
                          "bytes": T * (s.d_I * 4 + s.d_I + 4 + 4 * s.Dk),
                          "note": "per call, 20 calls per CUDA graph replay; not part of the metric's step"},
         "indexer_kl": indexer_kl_summary(kl_us, T, s, kl_valid, hbm, hbm_src),
+        **({"attn_backward": attn_backward_summary(bwd[0], T, s, bwd[1], hbm, hbm_src)} if bwd else {}),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(wt0, wt1),
     }
@@ -477,6 +505,26 @@ def indexer_kl_summary(us, T, s, valid, hbm, hbm_src):
             "algorithmic_bytes_per_call": algo, "flops": 2.0 * valid * s.H * s.Dk,
             "traffic": captured_traffic("indexer_kl_traffic.txt"),
             "note": "per call (loss and gradient), L2 flushed before each of 20 timed calls; "
+                    "not part of the metric's step"}
+
+
+def attn_backward_summary(us, T, s, valid, hbm, hbm_src):
+    """Per-call time of the sparse-attention backward against HBM bandwidth: each
+    call reads every selected latent row, the query, output-gradient and output
+    blocks, and adds into dq and into the selected rows of dkv (fp32, read and
+    written)."""
+    algo = (valid * (s.Dk * 2 + 2 * s.Dk * 4)          # row gathered, its dkv row read and written
+            + T * s.H * (s.Dk * 2 + 2 * s.Dv * 2 + 4)   # q, dO, o, lse
+            + T * s.H * s.Dk * 4 * 2                     # dq read and written
+            + T * s.k * 4)                               # the selection
+    gbs = algo / (us * 1e-6) / 1e9
+    flops = 2.0 * valid * s.H * (3 * s.Dk + 2 * s.Dv)     # S, dP, dKV (two terms), dQ
+    return {"us": us, "rows": T, "k": s.k, "api": "dsa_sparse_mqa_attn_backward", "kernel": "attn_bwd_kernel",
+            "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_call": algo, "flops": flops,
+            "note": "per call (delta kernel included), L2 flushed before each of 10 timed calls; "
                     "not part of the metric's step"}
 
 
