@@ -41,3 +41,11 @@ def test_indexer_loss_bytes_match_the_profile_count():
     assert out["algorithmic_bytes_per_call"] == 40_509_504
     assert abs(out["frac"] - out["achieved"] / 6559.0) < 1e-12
     assert out["bound"] == "hbm" and out["unit"] == "GB/s"
+
+
+def test_attention_backward_bytes_by_hand():
+    # 32768 slots x (1152 + 2 x 2304) + 16 rows x 128 heads x (1152 + 2 x 1024 + 4)
+    # + dq read and written 16 x 128 x 576 x 8 + the selection 16 x 2048 x 4
+    s = W.PAGED_DECODE_128K
+    out = bench.attn_backward_summary(50.0, 16, s, 16 * 2048, 6559.0, "measured")
+    assert out["algorithmic_bytes_per_call"] == 188_743_680 + 6_561_792 + 9_437_184 + 131_072
