@@ -172,12 +172,12 @@ dsa_status dsa_cache_append(const void *k_new, dsa_dtype k_dt, const void *kv_ne
  * lse is the attention's log-sum-exp per head over the same S_t, as
  * dsa_sparse_mqa_attn returns it, so that p_t is the heads' mean attention.
  *   q, kv, idx, lay   as for dsa_sparse_mqa_attn (bf16, H = 128, Dk = 576;
- *                     positions in S_t distinct; kv 16-byte aligned)
+ *                     positions in S_t distinct; q and kv 16-byte aligned)
  *   lse      device float32 [T][H];  scores device float32 [T][ld], ld >= the cache extent
  *   loss     device float32 [T] (written: zeroed, then the row's slot ranges add their
  *            terms with atomic adds, so its last bits may differ between runs)
  *   grad     device float32 [T][k], or NULL to skip the gradient
- * q, idx, lse, scores, loss and grad 4-byte aligned. Index errors are device
+ * idx, lse, scores, loss and grad 4-byte aligned. Index errors are device
  * check failures as in dsa_sparse_mqa_attn; a row with an empty S_t gets loss 0.
  */
 dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt,

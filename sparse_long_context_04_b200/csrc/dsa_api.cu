@@ -346,10 +346,10 @@ dsa_status dsa_indexer_kl(const void *q, const void *kv, dsa_dtype dt, int T, in
   const long long capn = L.page_size ? (long long)L.max_pages * L.page_size : L.n_max;
   if (ld < capn) return DSA_ERR_INVALID_ARG;
   if (dt != DSA_BF16 || H != 128 || Dk != 576 || k > 16384) return DSA_ERR_UNSUPPORTED;
-  const uintptr_t a4 = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(lse) |
-                       reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(loss) |
-                       reinterpret_cast<uintptr_t>(grad) | reinterpret_cast<uintptr_t>(idx);
-  if ((a4 & 3u) != 0 || !a16(kv)) return DSA_ERR_INVALID_ARG;
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(scores) |
+                       reinterpret_cast<uintptr_t>(loss) | reinterpret_cast<uintptr_t>(grad) |
+                       reinterpret_cast<uintptr_t>(idx);
+  if ((a4 & 3u) != 0 || !a16(q) || !a16(kv)) return DSA_ERR_INVALID_ARG;  // q is read by TMA
   if (T == 0) return DSA_OK;
   ErrCtx e;
   int sms;

@@ -117,8 +117,8 @@ def test_indexer_kl_rejects_bad_arguments_without_gpu(lib):
     A = 4096
     lay = _decode_layout()          # contiguous, n_max 256
 
-    def kl(dt=D.DSA_BF16, H=128, Dk=576, k=2048, ld=256, kv=A, loss=A, grad=A, lse=A, T=2):
-        return lib.dsa_indexer_kl(vp(A), vp(kv), dt, T, H, Dk, ctypes.c_float(0.1), vp(A), k, ctypes.byref(lay),
+    def kl(dt=D.DSA_BF16, H=128, Dk=576, k=2048, ld=256, q=A, kv=A, loss=A, grad=A, lse=A, T=2):
+        return lib.dsa_indexer_kl(vp(q), vp(kv), dt, T, H, Dk, ctypes.c_float(0.1), vp(A), k, ctypes.byref(lay),
                                   vp(lse), vp(A), ld, vp(loss), vp(grad), None)
 
     assert kl(loss=None) == D.DSA_ERR_INVALID_ARG
@@ -128,6 +128,7 @@ def test_indexer_kl_rejects_bad_arguments_without_gpu(lib):
     assert kl(H=64) == D.DSA_ERR_UNSUPPORTED
     assert kl(k=16385) == D.DSA_ERR_UNSUPPORTED
     assert kl(kv=A + 8) == D.DSA_ERR_INVALID_ARG                          # latent rows in 16-byte pieces
+    assert kl(q=A + 4) == D.DSA_ERR_INVALID_ARG                           # the query block is read by TMA
     assert kl(grad=A + 2) == D.DSA_ERR_INVALID_ARG
     assert kl(T=3) == D.DSA_ERR_INVALID_ARG                               # decode: one row per sequence
 
