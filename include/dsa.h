@@ -109,6 +109,32 @@ dsa_status dsa_topk(const float *scores, long long ld, int T, int k,
                     const dsa_seq_layout *lay, int *idx, void *stream);
 
 /*
+ * Stage 2 from a filtered candidate list: the finishing half of an indexer ->
+ * top-k that does not write its full score rows. Same result, order and tie rule
+ * as dsa_topk over the row's complete scores.
+ * Order key of a score x (the rule dsa_topk ranks by): 0 for NaN; otherwise, with
+ * u the bits of x and -0 taken as +0, u | 0x80000000 for x >= 0 and ~u for x < 0.
+ * The bin of x is its order key >> 20 (4096 bins).
+ *   hist    device uint32 [T][4096]: for each row, how many of its scores
+ *           s = 0..pos_t fall in each bin (all pos_t + 1 of them)
+ *   score, pos  device float32 / int32 [T][cap]: each row's candidates, any order,
+ *           each position at most once. Every position whose bin is at or above
+ *           the row's threshold bin (the bin of its k-th best key) must be there;
+ *           a producer gets this by keeping each key whose bin is at or above any
+ *           lower bound of the threshold bin, e.g. one read from the row's
+ *           histogram so far (the highest bin with at least k keys at or above).
+ *           Candidates below the threshold bin are ignored.
+ *   count   device int32 [T]: candidates per row (<= cap)
+ *   idx     device int32 [T][k], as dsa_topk writes it
+ * Rows up to 262144 keys; k >= 1. A histogram or candidate list that breaks the
+ * rules above (counts that disagree, a position out of range) is a device check
+ * failure and the row is written as -1.
+ */
+dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const int *count,
+                                    long long cap, const unsigned *hist, int T, int k,
+                                    const dsa_seq_layout *lay, int *idx, void *stream);
+
+/*
  * Stage 3 — sparse MQA attention over the selected latent rows.
  * For row t and head h, over the selected set S_t = {idx[t*k+i] >= 0}:
  *   z_s = softmax_scale * (q[t,h,:] . kv[s,:])   (Dk dims),

@@ -279,6 +279,22 @@ size_t dsa_sparse_mqa_attn_workspace_size(int T, int H, int Dv, int k, dsa_dtype
   return attn_ws(T, k, dt, sms);
 }
 
+dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const int *count, long long cap,
+                                    const unsigned *hist, int T, int k, const dsa_seq_layout *lay, int *idx,
+                                    void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  if (!score || !pos || !count || !hist || !idx || k < 1 || cap < 1) return DSA_ERR_INVALID_ARG;
+  if (capacity(L) > 262144) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_topk_candidates(score, pos, count, cap, hist, T, k, L, idx, e,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt, int T, int H, int Dk, int Dv,
                                float softmax_scale, const int *idx, int k, const dsa_seq_layout *lay, void *out,
                                float *lse, void *workspace, size_t ws_bytes, void *stream) {

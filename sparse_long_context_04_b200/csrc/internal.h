@@ -92,6 +92,13 @@ cudaError_t launch_attn_bwd(const void *q, const void *kv, int T, float scale, c
                             const Layout &L, const void *out, const void *dout, const float *lse, float *dq,
                             float *dkv, void *ws, const ErrCtx &e, cudaStream_t stream);
 
+// top-k from a filtered candidate list and the rows' complete 12-bit histograms
+// (topk_candidates.cu)
+size_t topk_candidates_smem();
+cudaError_t launch_topk_candidates(const float *score, const int *pos, const int *count, long long cap,
+                                   const unsigned *hist, int T, int k, const Layout &L, int *idx, const ErrCtx &e,
+                                   cudaStream_t stream);
+
 // indexer loss on the selected set and its gradient (indexer_kl.cu): bf16, H = 128, Dk = 576
 cudaError_t launch_indexer_kl(const void *q, const void *kv, int T, float scale, const int *idx, int k,
                               const float *lse, const float *scores, long long ld, const Layout &L, float *loss,

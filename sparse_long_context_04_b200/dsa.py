@@ -58,7 +58,7 @@ EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
            "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site",
            "dsa_cache_append", "dsa_indexer_kl", "dsa_sparse_mqa_attn_backward",
-           "dsa_sparse_mqa_attn_backward_workspace_size")
+           "dsa_sparse_mqa_attn_backward_workspace_size", "dsa_topk_from_candidates")
 
 
 def lib() -> ctypes.CDLL:
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         vp, i, ll, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
         L.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, i, vp, i, i, i, ctypes.POINTER(SeqLayout), vp, ll, vp]
         L.dsa_topk.argtypes = [vp, ll, i, i, ctypes.POINTER(SeqLayout), vp, vp]
+        L.dsa_topk_from_candidates.argtypes = [vp, vp, vp, ll, vp, i, i, ctypes.POINTER(SeqLayout), vp, vp]
+        L.dsa_topk_from_candidates.restype = i
         L.dsa_sparse_mqa_attn_workspace_size.argtypes = [i, i, i, i, i]
         L.dsa_sparse_mqa_attn_workspace_size.restype = sz
         L.dsa_sparse_mqa_attn.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i, ctypes.POINTER(SeqLayout),
@@ -164,6 +166,15 @@ def dsa_topk(scores, k, layout: Layout, idx, T=None, stream=None):
     s = lib().dsa_topk(_p(scores), int(scores.stride(0)), int(T), int(k), ctypes.byref(layout.c), _p(idx),
                        _stream(stream))
     _check(s, "dsa_topk")
+
+
+def dsa_topk_from_candidates(score, pos, count, hist, k, layout: Layout, idx, stream=None):
+    """Top-k of each row from its candidate list and complete 12-bit histogram
+    (see include/dsa.h): score/pos [T][cap], count [T], hist [T][4096]."""
+    T, cap = (int(x) for x in score.shape)
+    s = lib().dsa_topk_from_candidates(_p(score), _p(pos), _p(count), cap, _p(hist), T, int(k),
+                                       ctypes.byref(layout.c), _p(idx), _stream(stream))
+    _check(s, "dsa_topk_from_candidates")
 
 
 def dsa_sparse_mqa_attn_workspace_size(T, H, Dv, k, dtype) -> int:

@@ -155,3 +155,21 @@ def test_attention_backward_rejects_bad_arguments_without_gpu(lib):
     assert bwd(ws=A + 128) == D.DSA_ERR_WORKSPACE
     assert lib.dsa_sparse_mqa_attn_backward_workspace_size(2) == 1024
     assert lib.dsa_sparse_mqa_attn_backward_workspace_size(0) == 0
+
+
+def test_topk_from_candidates_rejects_bad_arguments_without_gpu(lib):
+    vp = ctypes.c_void_p
+    A = 4096
+    lay = _decode_layout()
+
+    def call(score=A, count=A, hist=A, k=2048, cap=256, T=2, n_max=256):
+        lay.n_max = n_max
+        return lib.dsa_topk_from_candidates(vp(score), vp(A), vp(count), cap, vp(hist), T, k, ctypes.byref(lay),
+                                            vp(A), None)
+
+    assert call(hist=None) == D.DSA_ERR_INVALID_ARG
+    assert call(count=None) == D.DSA_ERR_INVALID_ARG
+    assert call(k=0) == D.DSA_ERR_INVALID_ARG
+    assert call(cap=0) == D.DSA_ERR_INVALID_ARG
+    assert call(T=3) == D.DSA_ERR_INVALID_ARG                             # decode: one row per sequence
+    assert call(n_max=262145) == D.DSA_ERR_UNSUPPORTED                    # rows up to 262144 keys

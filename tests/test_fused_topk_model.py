@@ -1,14 +1,18 @@
-"""Exactness of the planned fused indexer -> top-k selection, checked on a numpy
-model of its steps (no GPU, no kernel): keys arrive tile by tile from several
-CTAs in an arbitrary interleaving; each tile is filtered against a lower bound
-on the row's k-th largest key that may be stale by any number of tiles (the
-floor of the highest 12-bit radix bin with at least k keys at or above it in the
-row's histogram so far); the survivors are appended in arrival order; a final
-step takes the threshold bin from the complete histogram, ranks that bin's
-candidates by (key descending, position ascending) and emits the positions in
-ascending order. The result must equal the oracle's top-k for every row,
-including ties, -0 against +0, infinities, NaN, rows shorter than k and score
-orders that defeat the filter (scores rising with position)."""
+"""Exactness of the fused indexer -> top-k selection, checked on numpy models
+(no GPU, no kernel).
+
+The producer-and-finisher model: keys arrive tile by tile from several CTAs in an
+arbitrary interleaving; each tile is filtered against a lower bound on the row's
+k-th largest key that may be stale by any number of tiles (the floor of the
+highest 12-bit radix bin with at least k keys at or above it in the row's
+histogram so far); the survivors are appended in arrival order; a final step
+takes the threshold bin from the complete histogram, ranks that bin's candidates
+by (key descending, position ascending) and emits the positions in ascending
+order. The finishing kernel's own steps are then emulated digit by digit (two
+10-bit key digits and two 9-bit position digits inside the threshold bin). Both
+must equal the oracle's top-k for every row, including ties, -0 against +0,
+infinities, NaN, rows shorter than k and score orders that defeat the filter
+(scores rising with position)."""
 import numpy as np
 import pytest
 
@@ -103,3 +107,81 @@ def test_candidates_are_few_on_unordered_scores():
     got, ncand = fused_select(x, 2048, 9, rng)
     assert np.array_equal(got, O.topk_row(x, 2048))
     assert ncand < 0.25 * x.size, ncand
+
+
+# ---------------------------------------------------------------------------
+# The finishing kernel's own steps (topk_candidates_kernel): the threshold bin
+# from the histogram, two 10-bit key digits and two 9-bit position digits inside
+# it, and the bitmap of selected positions, emulated digit by digit.
+
+def _find_digit(cnt, need, from_top):
+    before = 0
+    for d in (range(1023, -1, -1) if from_top else range(1024)):
+        if before < need <= before + cnt[d]:
+            return d, before
+        before += cnt[d]
+    raise AssertionError("no digit")
+
+
+def kernel_steps(x, hist, cand, k):
+    n = x.size
+    m = min(k, n)
+    above, B, above_b = 0, None, None
+    for b in range(4095, -1, -1):
+        if above < m <= above + hist[b]:
+            B, above_b = b, above
+        above += hist[b]
+    keys = order_key(x)
+    chosen = np.zeros(n, bool)
+    ties = []
+    for s in cand:
+        key = int(keys[s])
+        if key >> 20 > B:
+            chosen[s] = True
+        elif key >> 20 == B:
+            ties.append((key, int(s)))
+    assert chosen.sum() == above_b and len(ties) == hist[B]
+    need_ties = m - above_b
+    kstar, pstar = 0, (1 << 18) - 1
+    if need_ties < len(ties):
+        prefix, need = B << 20, need_ties
+        for shift, pmask in ((10, 0xFFF00000), (0, 0xFFFFFC00)):
+            cnt = np.zeros(1024, np.int64)
+            for key, _ in ties:
+                if key & pmask == prefix:
+                    cnt[(key >> shift) & 1023] += 1
+            d, rem = _find_digit(cnt, need, True)
+            prefix |= d << shift
+            need -= rem
+        kstar = prefix
+        for p in range(2):
+            shift = 9 if p == 0 else 0
+            cnt = np.zeros(1024, np.int64)
+            for key, s in ties:
+                if key == kstar and (p == 0 or s >> 9 == pstar >> 9):
+                    cnt[(s >> shift) & 511] += 1
+            d, rem = _find_digit(cnt, need, False)
+            pstar = (d << 9) | 511 if p == 0 else (pstar & ~511) | d
+            need -= rem
+    for key, s in ties:
+        if need_ties >= len(ties) or key > kstar or (key == kstar and s <= pstar):
+            chosen[s] = True
+    out = np.full(k, -1, np.int32)
+    sel = np.nonzero(chosen)[0]
+    assert sel.size == m
+    out[:m] = sel
+    return out
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_finishing_kernel_steps_equal_the_oracle(seed):
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(30):
+        x = _rows(rng)
+        k = int(rng.choice([1, 7, 64, 2048]))
+        bins = (order_key(x) >> 20).astype(np.int64)
+        hist = np.bincount(bins, minlength=4096)
+        bound = bound_bin(hist, k) if rng.random() < 0.5 else 0
+        cand = np.nonzero(bins >= bound)[0]
+        rng.shuffle(cand)
+        assert np.array_equal(kernel_steps(x, hist, cand, k), O.topk_row(x, k)), (x.size, k)
