@@ -173,10 +173,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill FP8 indexer measurement")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the sparse-attention backward on the step's selection")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the sparse-attention backward on the step's selection")
     ap.add_argument("--all-configs", action="store_true",
                     help="time every workload (stages, forward, roofline fractions), one JSON line each")
+    ap.add_argument("--only", default=None,
+                    help="with --all-configs: time this one workload (by name) only")
     ap.add_argument("--len-range", type=int, nargs=2, default=None,
                     help="override the context-length range (profiling on a smaller case)")
     args = ap.parse_args()
@@ -202,7 +204,7 @@ def main():
 
     if args.all_configs:
         if rank == 0:
-            all_configs(dev, G, D, W)
+            all_configs(dev, G, D, W, only=args.only)
         X.finish()
         return
 
@@ -366,7 +368,7 @@ def main():
     # ---- sparse-attention backward on the last step's selection and output (a
     # training-side call, outside the metric's step), L2 flushed before each call
     bwd = None
-    if args.backward:
+    if not args.no_backward:
         g = torch.Generator(device=dev).manual_seed(4321)
         dout = torch.randn((T, s.H, s.Dv), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
         dq = torch.zeros((T, s.H, s.Dk), dtype=torch.float32, device=dev)
@@ -417,8 +419,10 @@ def main():
     del graph
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during the cache write")
-    # ---- prefill FP8 indexer (tensor-bound): the 8K-token causal prefill
-    pf = prefill_indexer(args, dev, G, D, W) if not args.no_prefill else None
+    # ---- prefill FP8 indexer (tensor-bound): the 8K-token causal prefill, against
+    # the dense FP8 peak measured here
+    fp8_tf = measure_fp8_peak(dev) if not args.no_prefill else None
+    pf = prefill_indexer(args, dev, G, D, W, fp8_measured=fp8_tf) if not args.no_prefill else None
     sampler.stop_flag.set()
     sampler.join()
     if D.dsa_get_device_error() != D.DSA_OK:
@@ -470,6 +474,8 @@ def main():
                                "algorithmic_bytes": ab["topk"] + ab["attn"]},
         "step_roofline": {"achieved": step_gbs, "frac": step_gbs / hbm, "algorithmic_bytes": sum(ab.values())},
         "fp8_indexer_prefill": pf,
+        "fp8_peak_tflops": {"measured": fp8_tf, "datasheet": FP8_DATASHEET_TFLOPS,
+                            "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10, CUDA events"},
         "e2e": {"value": X.job_rate(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "api": "dsa_forward",
@@ -528,10 +534,51 @@ def attn_backward_summary(us, T, s, valid, hbm, hbm_src):
                     "not part of the metric's step"}
 
 
-def prefill_indexer(args, dev, G, D, W, reps=20):
+FP8_DATASHEET_TFLOPS = 4500.0   # dense e4m3, per GPU (context only)
+
+
+def measure_fp8_peak(dev, n=8192, reps=10):
+    """Dense e4m3 x e4m3 -> bf16 GEMM throughput of torch._scaled_mm at n^3
+    (2 n^3 flop), best of `reps` CUDA-event-timed calls after warm-up: the same
+    method as the measured bf16 peak, for the FP8 roofline. None if the call is
+    unavailable."""
+    try:
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize(dev)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+
+
+def fp8_peak(measured):
+    """(peak TFLOP/s, where it comes from) for the FP8 roofline."""
+    if measured:
+        return measured, "measured in this run: torch._scaled_mm e4m3 8192^3, best of 10"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 2 * float(json.load(f)["bf16_tflops"]), "estimate: 2x measured bf16 burst (nominal ratio)"
+    except Exception:
+        return 2 * 1590.0, "estimate: 2x fallback bf16"
+
+
+def prefill_indexer(args, dev, G, D, W, reps=20, fp8_measured=None):
     """Event-timed FP8 indexer over the causal 8192-token prefill: 16384 flop per
-    (query, earlier key) pair, against the FP8 dense peak (2x the measured bf16
-    burst, the nominal ratio; FP8 is not in the measured-peaks file)."""
+    (query, earlier key) pair, against the dense FP8 peak measured in the same run
+    (and, for context, the 4.5 PFLOP/s datasheet figure)."""
     spec = W.PREFILL_8K
     inp = W.make_inputs(spec)
     dc = G.to_device(inp, dev)
@@ -550,18 +597,13 @@ def prefill_indexer(args, dev, G, D, W, reps=20):
     pairs = L * (L + 1) // 2
     flops = pairs * 2 * spec.H_I * spec.d_I
     tf = flops / (ms / 1e3) / 1e12
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            bf16 = float(json.load(f)["bf16_tflops"])
-        src = "2x measured bf16 burst (nominal fp8/bf16 ratio)"
-    except Exception:
-        bf16, src = 1590.0, "2x fallback bf16"
-    peak = 2 * bf16
+    peak, src = fp8_peak(fp8_measured)
     return {"workload": spec.name, "us": ms * 1e3, "pairs": pairs, "tflops": tf, "peak_tflops": peak,
-            "frac": tf / peak, "peak_source": src, "kernel": "indexer_fp8_kernel (prefill, N=256)"}
+            "frac": tf / peak, "peak_source": src, "frac_of_datasheet": tf / FP8_DATASHEET_TFLOPS,
+            "datasheet_tflops": FP8_DATASHEET_TFLOPS, "kernel": "indexer_fp8_kernel (prefill, N=256)"}
 
 
-def all_configs(dev, G, D, W):
+def all_configs(dev, G, D, W, only=None):
     """Every workload once: per-stage CUDA-event times (each stage called on its own),
     the composed dsa_forward, tokens/s and each stage against its roofline (the larger
     of bytes / measured HBM and flops / the dtype's peak). One JSON line per workload."""
@@ -571,9 +613,11 @@ def all_configs(dev, G, D, W):
             bf16 = float(json.load(f)["bf16_tflops"])
     except Exception:
         bf16 = 1590.0
-    fp8 = 2 * bf16
+    fp8, fp8_src = fp8_peak(measure_fp8_peak(dev))
     for spec, reps in ((W.TINY, 20), (W.DECODE_32K, 50), (W.PREFILL_8K, 5), (W.PREFILL_2X32K, 2),
                        (W.PAGED_DECODE_128K, 50)):
+        if only and spec.name != only:
+            continue
         inp = W.make_inputs(spec)
         dc = G.to_device(inp, dev)
         T, s = dc.T, spec
@@ -631,7 +675,7 @@ def all_configs(dev, G, D, W):
             line["roofline_ms"] = roof
             line["frac"] = {k: roof[k] / ms[k] for k in roof}
             line["forward_frac"] = sum(roof.values()) / fwd_ms
-            line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": bf16, "fp8_tflops": fp8}
+            line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": bf16, "fp8_tflops": fp8, "fp8_source": fp8_src}
         print(json.dumps(line), flush=True)
         del dc, scores, idx, out, lse, ws, fw
         torch.cuda.empty_cache()

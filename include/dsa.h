@@ -252,13 +252,19 @@ dsa_status dsa_sparse_mqa_attn_backward(const void *q, const void *kv, dsa_dtype
  * variable, so this call never allocates device memory. It is for callers that
  * may not allocate: code running under a host framework that has reserved all
  * device memory up front, or a serving loop where cudaMalloc's implicit device
- * synchronisation is not allowed. Every GPU that loads the library holds the
- * 40 MiB until the process exits.
+ * synchronisation is not allowed. The 40 MiB are device memory of the library's
+ * module: under CUDA's lazy module loading they are taken when the module is
+ * first loaded on a device (at the latest by the first call of this entry point
+ * there) and held until the process exits.
  *   - A call needs T * ceil(k/256) * 132096 bytes of scratch (39 decode rows at
  *     k = 2048 fit); larger calls return DSA_ERR_TOO_LARGE and launch nothing.
  *   - The first call on each device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     that device current) and caches it per device index for the life of the
+ *     process (the primary context is assumed to live that long: after a
+ *     cudaDeviceReset the cached address is stale). Make that first call before
+ *     the caller reserves its device memory and before any stream capture. A
+ *     call with T = 0 (a prefill layout whose cu_q ranges are all empty) does
+ *     only this set-up and launches nothing: a cheap first call.
  *   - All calls share the one array: calls whose kernels may overlap on the GPU
  *     (other streams, other host threads) race on it and must be serialised by
  *     the caller. Nothing in it needs to start at zero.

@@ -529,6 +529,11 @@ cudaError_t scratch_address(void **out) {
 
 size_t attn_bf16_scratch_limit() { return kScratchBytes; }
 
+cudaError_t attn_bf16_scratch_setup() {
+  void *scratch = nullptr;
+  return scratch_address(&scratch);
+}
+
 size_t attn_bf16_scratch_bytes(int T, int k) {
   const AttnPlan pl = attn_bf16_plan(T, k, 0);
   return (size_t)T * part_bytes_per_row(pl.splits);

@@ -319,11 +319,11 @@ dsa_status dsa_sparse_mqa_attn_noalloc(const void *q, const void *kv, dsa_dtype 
   s = check_attn(q, kv, dt, H, Dk, Dv, idx, k, L, out);
   if (s != DSA_OK) return s;
   if (dt != DSA_BF16) return DSA_ERR_UNSUPPORTED;
-  if (T == 0) return DSA_OK;
   if (dsa::attn_bf16_scratch_bytes(T, k) > dsa::attn_bf16_scratch_limit()) return DSA_ERR_TOO_LARGE;
   ErrCtx e;
   int sms;
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  if (T == 0) return from_cuda(dsa::attn_bf16_scratch_setup());  // set-up only: a cheap first call
   return from_cuda(dsa::launch_attn_bf16_noalloc(q, kv, T, softmax_scale, idx, k, L, out, lse, e, sms,
                                                  static_cast<cudaStream_t>(stream)));
 }

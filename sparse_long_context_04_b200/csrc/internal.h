@@ -71,6 +71,8 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
 // same attention with its partials in the library's static scratch array
 size_t attn_bf16_scratch_bytes(int T, int k);
 size_t attn_bf16_scratch_limit();
+// looks up the scratch array's address on the current device (first use per device)
+cudaError_t attn_bf16_scratch_setup();
 cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float scale, const int *idx, int k,
                                      const Layout &L, void *out, float *lse, const ErrCtx &e, int num_sms,
                                      cudaStream_t stream);
