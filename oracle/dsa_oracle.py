@@ -1,423 +1,383 @@
-"""CPU oracle for the DeepSeek Sparse Attention (DSA) hot path.
+"""Python access to the CPU oracle of the DSA hot path (oracle/dsa_oracle.cpp).
 
-TEST INFRASTRUCTURE ONLY. This module is imported by the tests, by the smoke
-check and by the benchmark's CPU-baseline leg; the product path never calls it.
-It is a plain, slow, float64 statement of what the three stages compute. It
-shares no code with the CUDA library and imports nothing from it.
+TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's CPU
+legs use it; the product path never does. Every number here is computed by the
+plain C++ program (double precision, one query row at a time, rows spread over
+std::threads); this module only converts numpy arrays and the workload dicts
+of tests/case_utils.py into its arguments. It shares nothing with the CUDA
+library and imports nothing from it.
 
-Sources (the DeepSeek-V3.2-Exp pages; none prints an equation, so each stage is
-written from the words):
-  [jdon-indexer]   jdon.com "DeepSeek-V3.2-Exp", paragraph introducing the
-                   lightning indexer: light enough for FP8, very few heads, scores
-                   each query token against each earlier token with a weighted
-                   sum of ReLU-activated dot products.
-  [jdon-matchmake] same page, the "matchmaking" analogy paragraph: ReLU applied to
-                   the q_I/k_I meeting score, w_I as the weight, the highest scores
-                   go into the top-k set; main attention cost O(L^2) -> O(L*k).
-  [jdon-sparse]    same page, sparse-training paragraph: each query keeps only the
-                   2048 (K = 2048) highest-scoring earlier tokens.
-  [jdon-select]    same page, fine-grained selection paragraph: only the k chosen
-                   key/value entries take part; the output hidden state is u_t.
-  [jdon-causal]    same page, opening paragraph on cost: every token otherwise
-                   attends to all tokens before it (O(L^2)).
-  [openi-mla]      openi.cn "DeepSeek-V3.2", technical section, items on the
-                   lightning indexer (scores between the query token and earlier
-                   tokens), token selection (top-k value entries) and MLA in MQA
-                   mode (one value entry shared by many queries).
-  [mundobytes-run] mundobytes.com run guide: the serving command uses page size 64.
-  [mundobytes-kernels] same page, open-kernels paragraph: the indexer kernels are
-                   published in a paged version.
-
-Readings taken where the pages are silent:
-  * I[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]), ReLU per head before the
-    weighted sum; the FP8 per-token scales multiply the dequantised vectors.
-  * causal set s <= pos_t, inclusive of the query's own position.
-  * top-k order: score descending, then index ascending; -0 == +0; NaN lowest;
-    emitted in ascending index order, padded with -1 when pos_t + 1 < k.
-  * attention: key = full latent row (Dk dims), value = its first Dv dims, one
-    row shared by all heads; plain softmax with a caller-given scale, no sink.
+The definitions it follows, and the readings taken where the DeepSeek-V3.2-Exp
+pages are silent, are stated in oracle/dsa_oracle.cpp beside each function:
+  * I[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]) for s <= pos_t (jdon.com
+    "DeepSeek-V3.2-Exp", lightning-indexer and matchmaking paragraphs);
+  * the min(k, pos_t + 1) best positions under (score desc, position asc),
+    ascending, -1 padded (same page, sparse-training and selection paragraphs);
+  * per-head softmax attention over the selected latent rows, key = the whole
+    row, value = its first Dv values (openi.cn "DeepSeek-V3.2", MLA-in-MQA item).
 """
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
+
+from . import build_oracle
+
+_lib = None
+_D = ctypes.POINTER(ctypes.c_double)
+_F = ctypes.POINTER(ctypes.c_float)
+_I = ctypes.POINTER(ctypes.c_int32)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
+_U16 = ctypes.POINTER(ctypes.c_uint16)
+_V = ctypes.c_void_p
+
+
+class _Case(ctypes.Structure):
+    _fields_ = [
+        ("fp8", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int),
+        ("H_I", ctypes.c_int), ("d_I", ctypes.c_int), ("H", ctypes.c_int), ("Dk", ctypes.c_int),
+        ("Dv", ctypes.c_int), ("k", ctypes.c_int), ("softmax_scale", ctypes.c_double),
+        ("seq_lens", _V), ("pos", _V), ("row_seq", _V),
+        ("q_idx", _V), ("q_scale", _V), ("w", _V), ("q", _V),
+        ("page_size", ctypes.c_int), ("n_max", ctypes.c_int),
+        ("k_idx", _V), ("k_scale", _V), ("k_pages", _V), ("page_table", _V), ("max_pages", ctypes.c_int),
+        ("kv", _V),
+    ]
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build_oracle.build())
+        ll, i, d = ctypes.c_longlong, ctypes.c_int, ctypes.c_double
+        sig = {
+            "oracle_hardware_threads": ([], i),
+            "oracle_e4m3_value": ([ctypes.c_uint], d),
+            "oracle_bf16_value": ([ctypes.c_uint], d),
+            "oracle_decode_e4m3": ([_V, ll, _V], None),
+            "oracle_decode_bf16": ([_V, ll, _V], None),
+            "oracle_dequant": ([_V, ll, ll, _V, _V], None),
+            "oracle_encode_e4m3": ([_V, ll, _V], None),
+            "oracle_quantize_key_row": ([_V, i, _V, _V], None),
+            "oracle_indexer_row": ([_V, _V, _V, ll, i, i, _V], None),
+            "oracle_topk_row": ([_V, i, i, _V], None),
+            "oracle_topk_rows": ([_V, ll, _V, i, i, _V, i], None),
+            "oracle_sparse_attn_row": ([_V, _V, i, i, i, i, d, _V, _V], None),
+            "oracle_seq_keys": ([ctypes.POINTER(_Case), i, _V, _V], None),
+            "oracle_query_row": ([ctypes.POINTER(_Case), i, _V, _V, _V], None),
+            "oracle_indexer_rows": ([ctypes.POINTER(_Case), _V, i, _V, ll, i], None),
+            "oracle_attn_rows": ([ctypes.POINTER(_Case), _V, i, _V, _V, _V, i], None),
+            "oracle_forward_rows": ([ctypes.POINTER(_Case), _V, i, _V, ll, _V, _V, _V, i], None),
+            "oracle_cache_append": ([ctypes.POINTER(_Case), _V, _V, _V, _V, _V], None),
+            "oracle_indexer_kl_row": ([_V, _V, i, i, i, d, _V, _V, _V], d),
+            "oracle_attn_backward_row": ([_V, _V, i, i, i, i, d, _V, _V, _V], None),
+            "oracle_attn_backward_seq": ([_V, _V, ll, _V, i, i, i, i, i, d, _V, _V, _V], None),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def threads() -> int:
+    """Threads the oracle uses for many rows (the host's hardware threads)."""
+    return int(lib().oracle_hardware_threads())
+
+
+def _c(a, dtype):
+    """C-contiguous array of `dtype` (no copy when it already is one) and its address."""
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(_V)
+
+
+def _out(shape, dtype=np.float64):
+    a = np.zeros(shape, dtype=dtype)
+    return a, a.ctypes.data_as(_V)
+
 
 # ---------------------------------------------------------------------------
 # number formats
 
-
 def e4m3_value(byte: int) -> float:
-    """Value of one OCP FP8 E4M3 ("e4m3fn") byte, from the format definition:
-    1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 is
-    subnormal (m/8 * 2^-6); S.1111.111 is NaN; there is no infinity."""
-    s = (byte >> 7) & 1
-    e = (byte >> 3) & 0xF
-    m = byte & 0x7
-    if e == 0xF and m == 0x7:
-        return float("nan")
-    if e == 0:
-        mag = (m / 8.0) * 2.0 ** (-6)
-    else:
-        mag = (1.0 + m / 8.0) * 2.0 ** (e - 7)
-    return -mag if s else mag
+    """Value of one OCP FP8 E4M3 byte, from the format's bit fields."""
+    return float(lib().oracle_e4m3_value(int(byte)))
 
 
-E4M3_TABLE = np.array([e4m3_value(b) for b in range(256)], dtype=np.float64)
-
-
-def decode_e4m3(u8: np.ndarray) -> np.ndarray:
-    return E4M3_TABLE[np.asarray(u8, dtype=np.uint8)]
-
-
-def decode_bf16(bits: np.ndarray) -> np.ndarray:
-    """bfloat16 bit patterns -> float64 (bf16 is the top half of an IEEE binary32)."""
-    b = np.asarray(bits).view(np.uint16).astype(np.uint32) << 16
-    return b.view(np.float32).astype(np.float64)
-
-
-def dequant(u8_rows: np.ndarray, scale: np.ndarray) -> np.ndarray:
-    """x~ = s * dec(b) with one scale per leading row, in float64."""
-    x = decode_e4m3(u8_rows)
-    s = np.asarray(scale, dtype=np.float64).reshape((-1,) + (1,) * (x.ndim - 1))
-    return x * s
-
-
-# ---------------------------------------------------------------------------
-# stage 1: lightning indexer   [jdon-indexer], [jdon-matchmake], [openi-mla]
-
-
-def indexer_row(q_t: np.ndarray, w_t: np.ndarray, keys: np.ndarray) -> np.ndarray:
-    """Scores of one query token against `keys` (its causal prefix).
-
-    q_t  [H_I, d_I] float64: the token's indexer query heads (dequantised)
-    w_t  [H_I]      float64: the token's per-head weights
-    keys [n, d_I]   float64: indexer keys of positions 0..n-1 (dequantised)
-    returns I[s] = sum_j w_t[j] * max(0, q_t[j] . keys[s]),  s = 0..n-1
-    """
-    dots = keys @ q_t.T                      # [n, H_I]: q_I[t,j] . k_I[s]
-    return np.maximum(dots, 0.0) @ w_t       # ReLU per head, then the weighted sum
-
-
-# ---------------------------------------------------------------------------
-# stage 2: fine-grained token selection   [jdon-sparse], [jdon-select], [openi-mla]
-
-
-def topk_row(scores: np.ndarray, k: int) -> np.ndarray:
-    """Indices kept for one query row.
-
-    scores: float32 [n] — the row's scores over its causal prefix s = 0..n-1.
-    Returns int32 [k]: the m = min(k, n) indices that come first under the order
-    (score descending, index ascending), listed in ascending index order and
-    padded with -1. -0.0 and +0.0 compare equal; NaN ranks below every number.
-    """
-    v = np.asarray(scores, dtype=np.float32).astype(np.float64)
-    n = v.shape[0]
-    m = min(k, n)
-    idx = np.arange(n)
-    # primary key: -v ascending (NaN sorts last); secondary: index ascending
-    order = np.lexsort((idx, -v))
-    chosen = np.sort(order[:m])
-    out = np.full(k, -1, dtype=np.int32)
-    out[:m] = chosen
+def decode_e4m3(u8) -> np.ndarray:
+    a, p = _c(u8, np.uint8)
+    out, po = _out(a.shape)
+    lib().oracle_decode_e4m3(p, a.size, po)
     return out
 
 
+def decode_bf16(bits) -> np.ndarray:
+    """bfloat16 bit patterns -> float64."""
+    a, p = _c(np.asarray(bits).view(np.uint16), np.uint16)
+    out, po = _out(a.shape)
+    lib().oracle_decode_bf16(p, a.size, po)
+    return out
+
+
+def dequant(u8_rows, scale) -> np.ndarray:
+    """x~ = s * dec(b) with one scale per leading row, in float64."""
+    a, p = _c(u8_rows, np.uint8)
+    s, ps = _c(np.asarray(scale).reshape(-1), np.float32)
+    rows = s.size
+    out, po = _out(a.shape)
+    lib().oracle_dequant(p, rows, a.size // max(rows, 1), ps, po)
+    return out
+
+
+def encode_e4m3_rne(y) -> np.ndarray:
+    """e4m3 byte of the value nearest to each y (ties to even), saturating; NaN -> 0x7F."""
+    a, p = _c(y, np.float64)
+    out, po = _out(a.shape, np.uint8)
+    lib().oracle_encode_e4m3(p, a.size, po)
+    return out
+
+
+def quantize_key_row(x):
+    """(e4m3 bytes, fp32 scale) of one indexer key row, in fp32 arithmetic."""
+    a, p = _c(x, np.float32)
+    codes, pc = _out(a.shape, np.uint8)
+    sc = np.zeros(1, np.float32)
+    lib().oracle_quantize_key_row(p, a.size, pc, sc.ctypes.data_as(_V))
+    return codes, np.float32(sc[0])
+
+
 # ---------------------------------------------------------------------------
-# stage 3: sparse MQA attention over the latent rows   [jdon-select], [openi-mla]
+# the stages on plain arrays
+
+def indexer_row(q_t, w_t, keys) -> np.ndarray:
+    """I[s] = sum_j w_t[j] * max(0, q_t[j] . keys[s]) for q_t [H_I, d_I], w_t [H_I], keys [n, d_I]."""
+    q, pq = _c(q_t, np.float64)
+    w, pw = _c(w_t, np.float64)
+    k, pk = _c(keys, np.float64)
+    H_I, d_I = q.shape
+    n = k.shape[0] if k.ndim == 2 else 0
+    out, po = _out(n)
+    lib().oracle_indexer_row(pq, pw, pk, n, H_I, d_I, po)
+    return out
 
 
-def sparse_attn_row(q_t: np.ndarray, kv_rows: np.ndarray, Dv: int, scale: float):
-    """Attention of one query token over its selected latent rows.
+def topk_row(scores, k: int) -> np.ndarray:
+    """int32 [k]: the min(k, n) best positions (score desc, position asc; -0 == +0,
+    NaN lowest) of a float32 row, ascending, -1 padded."""
+    s, ps = _c(scores, np.float32)
+    out, po = _out(int(k), np.int32)
+    lib().oracle_topk_row(ps, s.size, int(k), po)
+    return out
 
-    q_t     [H, Dk] float64: the token's query heads
-    kv_rows [m, Dk] float64: the selected rows (key = whole row, value = first Dv dims)
-    returns (o [H, Dv], lse [H]) with z = scale * q.k, o = softmax(z) @ v,
-    lse = log sum exp z (natural log). Two-pass softmax.
-    """
-    z = scale * (q_t @ kv_rows.T)                   # [H, m]
-    zmax = z.max(axis=1, keepdims=True)
-    p = np.exp(z - zmax)
-    Z = p.sum(axis=1, keepdims=True)
-    o = (p @ kv_rows[:, :Dv]) / Z
-    lse = zmax[:, 0] + np.log(Z[:, 0])
+
+def topk_rows(scores, n, k: int, nthreads: int = 0) -> np.ndarray:
+    """topk_row of every row r of a float32 [R, ld] array over its first n[r] entries."""
+    s, ps = _c(scores, np.float32)
+    nn, pn = _c(n, np.int32)
+    R = nn.size
+    out, po = _out((R, int(k)), np.int32)
+    lib().oracle_topk_rows(ps, s.shape[1], pn, R, int(k), po, int(nthreads))
+    return out
+
+
+def sparse_attn_row(q_t, kv_rows, Dv: int, scale: float):
+    """(o [H, Dv], lse [H]): softmax attention of q_t [H, Dk] over kv_rows [m, Dk]."""
+    q, pq = _c(q_t, np.float64)
+    r, pr = _c(kv_rows, np.float64)
+    H, Dk = q.shape
+    m = r.shape[0] if r.ndim == 2 else 0
+    o, po = _out((H, int(Dv)))
+    lse, pl = _out(H)
+    lib().oracle_sparse_attn_row(pq, pr, m, H, Dk, int(Dv), float(scale), po, pl)
     return o, lse
 
 
-def dense_causal_mqa_online(q_t: np.ndarray, kv_prefix: np.ndarray, Dv: int, scale: float):
-    """Dense causal MQA for one token, written as a one-key-at-a-time online
-    softmax (a different algorithm from `sparse_attn_row`). Used to pin the
-    invariant that DSA with k >= L equals dense causal attention."""
-    H = q_t.shape[0]
-    m = np.full(H, -np.inf)
-    l = np.zeros(H)
-    acc = np.zeros((H, Dv))
-    for s in range(kv_prefix.shape[0]):
-        z = scale * (q_t @ kv_prefix[s])
-        m_new = np.maximum(m, z)
-        a = np.exp(m - m_new)
-        b = np.exp(z - m_new)
-        l = l * a + b
-        acc = acc * a[:, None] + b[:, None] * kv_prefix[s, :Dv][None, :]
-        m = m_new
-    return acc / l[:, None], m + np.log(l)
-
-
 # ---------------------------------------------------------------------------
-# logical views of the key caches (contiguous or paged)  [mundobytes-run]
+# workload dicts (tests/case_utils.py) -> the oracle's case description
+
+class _CaseRef:
+    """A _Case and the arrays it points into (kept alive together)."""
+
+    def __init__(self, case: dict):
+        fp8 = bool(case["fp8"])
+        keep = []
+
+        def arr(x, dtype):
+            if x is None:
+                return None
+            a = np.ascontiguousarray(x, dtype=dtype)
+            keep.append(a)
+            return a.ctypes.data_as(_V)
+
+        c = _Case()
+        c.fp8 = int(fp8)
+        kv = case["kv"]
+        seq = np.asarray(case["seq_lens"])
+        pos = np.asarray(case.get("pos", np.zeros(0, np.int32)))
+        c.B, c.T = int(seq.size), int(pos.size)
+        c.d_I = int(case["d_I"])
+        c.Dk = int(case.get("Dk", np.asarray(kv).shape[-1]))
+        c.H_I, c.H, c.Dv, c.k = (int(case.get(x, 0)) for x in ("H_I", "H", "Dv", "k"))
+        c.softmax_scale = float(case.get("softmax_scale", 1.0))
+        c.seq_lens, c.pos = arr(seq, np.int32), arr(pos, np.int32)
+        c.row_seq = arr(case.get("row_seq", np.zeros(0, np.int32)), np.int32)
+        qt = np.uint8 if fp8 else np.float32
+        c.q_idx = arr(case.get("q_idx"), qt)
+        c.q_scale = arr(case.get("q_scale"), np.float32) if fp8 else None
+        c.w = arr(case.get("w"), np.float32)
+        q = case.get("q")
+        c.q = arr(None if q is None else (np.asarray(q).view(np.uint16) if fp8 else q),
+                  np.uint16 if fp8 else np.float32)
+        c.page_size = int(case["page_size"])
+        if c.page_size:
+            pt = np.asarray(case["page_table"])
+            c.page_table = arr(pt, np.int32)
+            c.max_pages = int(pt.shape[1])
+            c.k_pages = arr(case["k_pages"], np.uint8)
+            c.n_max = 0
+        else:
+            c.k_idx = arr(case["k_idx"], np.uint8 if fp8 else np.float32)
+            c.k_scale = arr(case.get("k_scale"), np.float32) if fp8 else None
+            c.n_max = int(np.asarray(case["k_idx"]).shape[1])
+        c.kv = arr(np.asarray(kv).view(np.uint16) if fp8 else kv, np.uint16 if fp8 else np.float32)
+        self.c, self.keep = c, keep
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
 
 
 def seq_keys(case: dict, b: int):
-    """Float64 indexer keys [len_b, d_I] and latent rows [len_b, Dk] of sequence b,
-    in logical position order. A paged cache maps position s to page
-    page_table[b, s // P], slot s % P; an indexer page holds P key rows of d_I
-    bytes followed by P little-endian float32 scales."""
-    L = int(case["seq_lens"][b])
-    fp8 = case["fp8"]
-    P = case["page_size"]
-    if P == 0:
-        if fp8:
-            kI = dequant(case["k_idx"][b, :L], case["k_scale"][b, :L])
-            kv = decode_bf16(case["kv"][b, :L])
-        else:
-            kI = np.asarray(case["k_idx"][b, :L], dtype=np.float64)
-            kv = np.asarray(case["kv"][b, :L], dtype=np.float64)
-        return kI, kv
-    d_I = case["d_I"]
-    pos = np.arange(L)
-    page = case["page_table"][b, pos // P].astype(np.int64)
-    slot = pos % P
-    pages = case["k_pages"]
-    kbytes = pages[page[:, None], slot[:, None] * d_I + np.arange(d_I)[None, :]]
-    sbytes = pages[page[:, None], P * d_I + slot[:, None] * 4 + np.arange(4)[None, :]]
-    scale = np.ascontiguousarray(sbytes).view("<f4").reshape(L)
-    kI = dequant(kbytes, scale)
-    kv = decode_bf16(case["kv"][page, slot])
+    """Float64 indexer keys [len_b, d_I] and latent rows [len_b, Dk] of sequence b in
+    position order (paged caches read through the page table)."""
+    cr = _CaseRef(case)
+    L = int(np.asarray(case["seq_lens"])[b])
+    kI, pk = _out((L, cr.c.d_I))
+    kv, pv = _out((L, cr.c.Dk))
+    lib().oracle_seq_keys(cr.ref, int(b), pk, pv)
     return kI, kv
 
 
 def query_row(case: dict, t: int):
     """Float64 (indexer query heads [H_I, d_I], weights [H_I], query heads [H, Dk]) of row t."""
-    if case["fp8"]:
-        qI = dequant(case["q_idx"][t][None], case["q_scale"][t:t + 1])[0]
-        q = decode_bf16(case["q"][t])
-    else:
-        qI = np.asarray(case["q_idx"][t], dtype=np.float64)
-        q = np.asarray(case["q"][t], dtype=np.float64)
-    w = np.asarray(case["w"][t], dtype=np.float64)
+    cr = _CaseRef(case)
+    qI, p1 = _out((cr.c.H_I, cr.c.d_I))
+    w, p2 = _out(cr.c.H_I)
+    q, p3 = _out((cr.c.H, cr.c.Dk))
+    lib().oracle_query_row(cr.ref, int(t), p1, p2, p3)
     return qI, w, q
 
 
-# ---------------------------------------------------------------------------
-# whole path for chosen rows
+def _rows(rows):
+    r = np.ascontiguousarray(np.asarray(list(rows), dtype=np.int32))
+    return r, r.ctypes.data_as(_V)
 
 
-def forward_rows(case: dict, rows, keys_cache=None):
-    """Indexer -> top-k -> attention for query rows `rows` of `case`.
-
-    Returns {t: dict(scores=f64[pos+1], idx=int32[k], o=f64[H,Dv], lse=f64[H])}.
-    The selection runs on the oracle's own scores rounded to float32.
-    """
-    keys_cache = {} if keys_cache is None else keys_cache
-    out = {}
-    for t in rows:
-        b = int(case["row_seq"][t])
-        pos = int(case["pos"][t])
-        if b not in keys_cache:
-            keys_cache[b] = seq_keys(case, b)
-        kI, kv = keys_cache[b]
-        qI, w, q = query_row(case, t)
-        sc = indexer_row(qI, w, kI[:pos + 1])
-        idx = topk_row(sc.astype(np.float32), case["k"])
-        sel = idx[idx >= 0]
-        o, lse = sparse_attn_row(q, kv[sel], case["Dv"], case["softmax_scale"])
-        out[t] = dict(scores=sc, idx=idx, o=o, lse=lse)
-    return out
-
-
-def attn_rows_on_indices(case: dict, rows, idx_rows, keys_cache=None):
-    """Attention of `rows` recomputed on externally given index rows (e.g. a GPU's
-    selection): {t: (o [H,Dv], lse [H])}. Index -1 marks padding."""
-    keys_cache = {} if keys_cache is None else keys_cache
-    res = {}
-    for t, idx in zip(rows, idx_rows):
-        b = int(case["row_seq"][t])
-        if b not in keys_cache:
-            keys_cache[b] = seq_keys(case, b)
-        _, kv = keys_cache[b]
-        _, _, q = query_row(case, t)
-        idx = np.asarray(idx)
-        sel = idx[idx >= 0]
-        res[t] = sparse_attn_row(q, kv[sel], case["Dv"], case["softmax_scale"])
-    return res
-
-
-def indexer_rows(case: dict, rows, keys_cache=None):
+def indexer_rows(case: dict, rows, keys_cache=None, nthreads: int = 0):
     """Indexer scores of `rows` over their causal prefixes: {t: f64[pos+1]}."""
-    keys_cache = {} if keys_cache is None else keys_cache
+    cr = _CaseRef(case)
+    r, pr = _rows(rows)
+    pos = np.asarray(case["pos"])
+    ld = int(max((int(pos[t]) + 1 for t in r), default=1))
+    out, po = _out((r.size, ld))
+    lib().oracle_indexer_rows(cr.ref, pr, r.size, po, ld, int(nthreads))
+    return {int(t): out[i, :int(pos[t]) + 1] for i, t in enumerate(r)}
+
+
+def attn_rows_on_indices(case: dict, rows, idx_rows, keys_cache=None, nthreads: int = 0):
+    """Attention of `rows` recomputed on given selections (-1 = padding): {t: (o [H,Dv], lse [H])}."""
+    cr = _CaseRef(case)
+    r, pr = _rows(rows)
+    k = cr.c.k
+    ix = np.full((r.size, k), -1, np.int32)
+    for i, x in enumerate(idx_rows):
+        x = np.asarray(x, dtype=np.int32).reshape(-1)
+        ix[i, :x.size] = x
+    ix, pi = _c(ix, np.int32)
+    o, po = _out((r.size, cr.c.H, cr.c.Dv))
+    lse, pl = _out((r.size, cr.c.H))
+    lib().oracle_attn_rows(cr.ref, pr, r.size, pi, po, pl, int(nthreads))
+    return {int(t): (o[i], lse[i]) for i, t in enumerate(r)}
+
+
+def forward_rows(case: dict, rows, keys_cache=None, nthreads: int = 0, want_scores: bool = True):
+    """Indexer -> top-k (on the scores rounded to float32) -> attention for `rows`:
+    {t: dict(scores=f64[pos+1], idx=int32[k], o=f64[H,Dv], lse=f64[H])}."""
+    cr = _CaseRef(case)
+    r, pr = _rows(rows)
+    pos = np.asarray(case["pos"])
+    ld = int(max((int(pos[t]) + 1 for t in r), default=1))
+    sc, ps = _out((r.size, ld)) if want_scores else (None, None)
+    idx, pi = _out((r.size, cr.c.k), np.int32)
+    o, po = _out((r.size, cr.c.H, cr.c.Dv))
+    lse, pl = _out((r.size, cr.c.H))
+    lib().oracle_forward_rows(cr.ref, pr, r.size, ps, ld, pi, po, pl, int(nthreads))
     res = {}
-    for t in rows:
-        b = int(case["row_seq"][t])
-        pos = int(case["pos"][t])
-        if b not in keys_cache:
-            keys_cache[b] = seq_keys(case, b)
-        kI, _ = keys_cache[b]
-        qI, w, _ = query_row(case, t)
-        res[t] = indexer_row(qI, w, kI[:pos + 1])
+    for i, t in enumerate(r):
+        res[int(t)] = dict(scores=None if sc is None else sc[i, :int(pos[t]) + 1], idx=idx[i], o=o[i], lse=lse[i])
     return res
 
 
 # ---------------------------------------------------------------------------
-# cache write: one new token per query row into the paged caches
-#   [mundobytes-run] pages of 64 tokens; [mundobytes-kernels] mundobytes.com, the
-#   open-kernels paragraph: the indexer kernels come in a paged version;
-#   [jdon-indexer] the indexer keys are stored and scored in FP8.
-# Readings: one fp32 scale per key token, scale = max|x| / 448 in
-# fp32 (1 when the row is all zero); code = the e4m3 value nearest to x / scale
-# (fp32 division), ties to the even code, saturating at +-448, the sign kept
-# for values that round to zero.
+# cache write, indexer loss, attention backward
 
-E4M3_MAX = 448.0
-
-
-def encode_e4m3_rne(y: np.ndarray) -> np.ndarray:
-    """e4m3 byte of the representable value nearest to each y (ties to the even
-    code), saturating to +-448; NaN -> 0x7F. The non-negative codes 0x00..0x7E
-    are the format's finite magnitudes in increasing order, so rounding is a
-    search in that table."""
-    y = np.asarray(y, dtype=np.float64)
-    mags = E4M3_TABLE[:127]                      # codes 0x00 .. 0x7E, increasing
-    a = np.minimum(np.abs(y), E4M3_MAX)
-    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, 126)   # first magnitude >= a
-    lo = np.clip(hi - 1, 0, 126)
-    d_lo = a - mags[lo]
-    d_hi = mags[hi] - a
-    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0) & (hi != lo))
-    code = np.where(take_hi, hi, lo).astype(np.uint8)
-    code = np.where(np.signbit(y), code | 0x80, code).astype(np.uint8)
-    return np.where(np.isnan(y), np.uint8(0x7F), code).astype(np.uint8)
-
-
-def quantize_key_row(x: np.ndarray):
-    """(e4m3 bytes, fp32 scale) of one indexer key row, in the kernel's fp32
-    arithmetic: scale = float32(max|x|) / float32(448); y = float32(x) / scale."""
-    x32 = np.asarray(x, dtype=np.float32)
-    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
-    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32) if amax > 0 else np.float32(1.0)
-    y = (x32 / scale).astype(np.float32)
-    return encode_e4m3_rne(y), np.float32(scale)
-
-
-def cache_append(case: dict, k_new: np.ndarray, kv_new_bits: np.ndarray, k_pool: np.ndarray,
-                 kv_pool_bits: np.ndarray, k_scale: np.ndarray = None):
-    """Write row t's new indexer key (quantised) and latent row (bf16 bits, copied)
-    at the row's own position pos_t of its sequence. Returns updated copies.
-
-    Paged (page_size 64): k_pool uint8 [pages][8448] = [64 x d_I codes][64 fp32
-    scales]; kv_pool_bits uint16 [pages*64][Dk]. Contiguous: k_pool uint8
-    [B][n_max][d_I], k_scale float32 [B][n_max], kv_pool_bits [B][n_max][Dk]."""
-    k_pool = k_pool.copy()
-    kv_pool_bits = kv_pool_bits.copy()
-    k_scale = None if k_scale is None else k_scale.copy()
-    P = int(case["page_size"])
-    d_I = k_new.shape[1]
-    for t in range(k_new.shape[0]):
-        b = int(case["row_seq"][t])
-        pos = int(case["pos"][t])
-        codes, sc = quantize_key_row(k_new[t])
-        if P:
-            page = int(case["page_table"][b][pos // P])
-            slot = pos % P
-            k_pool[page, slot * d_I:(slot + 1) * d_I] = codes
-            k_pool[page, P * d_I + 4 * slot:P * d_I + 4 * slot + 4] = np.frombuffer(
-                np.float32(sc).tobytes(), dtype=np.uint8)
-            kv_pool_bits[page * P + slot] = kv_new_bits[t]
-        else:
-            k_pool[b, pos] = codes
-            k_scale[b, pos] = sc
-            kv_pool_bits[b, pos] = kv_new_bits[t]
+def cache_append(case: dict, k_new, kv_new_bits, k_pool, kv_pool_bits, k_scale=None):
+    """Write row t's new indexer key (quantised per token) and latent row (bf16 bits)
+    at its own position; returns updated copies (k_pool, kv_pool_bits, k_scale)."""
+    kn, pk = _c(k_new, np.float32)
+    kv_new = None if kv_new_bits is None else np.ascontiguousarray(np.asarray(kv_new_bits).view(np.uint16))
+    k_pool = np.array(k_pool, dtype=np.uint8, copy=True, order="C")
+    kv_pool_bits = np.array(np.asarray(kv_pool_bits).view(np.uint16), copy=True, order="C")
+    k_scale = None if k_scale is None else np.array(k_scale, dtype=np.float32, copy=True, order="C")
+    full = dict(fp8=True, seq_lens=np.zeros(1, np.int32), d_I=int(kn.shape[1]), kv=kv_pool_bits, k_pages=k_pool,
+                k_idx=k_pool, k_scale=k_scale)
+    full.update({x: case[x] for x in ("page_size", "row_seq", "pos", "page_table") if x in case})
+    cr = _CaseRef(full)
+    cr.c.T = int(kn.shape[0])
+    lib().oracle_cache_append(cr.ref, pk, None if kv_new is None else kv_new.ctypes.data_as(_V),
+                              k_pool.ctypes.data_as(_V), None if k_scale is None else k_scale.ctypes.data_as(_V),
+                              kv_pool_bits.ctypes.data_as(_V))
     return k_pool, kv_pool_bits, k_scale
 
 
-# ---------------------------------------------------------------------------
-# indexer loss (sparse stage)
-#   [jdon-warmup] jdon.com "DeepSeek-V3.2-Exp", warm-up paragraph: the indexer first
-#   copies how the main attention distributes its attention, trained with a KL
-#   divergence loss; [jdon-sparse-train] same page, sparse-training paragraph: the
-#   indexer and the main model are trained together with separated gradients, the
-#   indexer optimising only its own scoring loss.
-# Readings: the target is the main attention's distribution over the selected set,
-# averaged over the heads (each head's softmax sums to 1, so the mean is
-# L1-normalised); the indexer's distribution is the softmax of its scores over the
-# same set; loss = KL(target || indexer); the indexer's gradient is
-# softmax(I) - target, and no gradient reaches the attention inputs.
-
-def indexer_kl_row(q_t: np.ndarray, kv_rows: np.ndarray, scale: float, scores: np.ndarray):
-    """(loss, target p, d loss / d scores) for one query row over its selected rows.
-
-    q_t [H, Dk] and kv_rows [m, Dk] as float64 values, scores [m] the indexer
-    scores of the same m selected positions."""
-    z = scale * (np.asarray(q_t, np.float64) @ np.asarray(kv_rows, np.float64).T)   # [H, m]
-    z = z - z.max(axis=1, keepdims=True)
-    a = np.exp(z)
-    a /= a.sum(axis=1, keepdims=True)            # each head's attention over the selected set
-    p = a.mean(axis=0)                           # target: mean over heads, sums to 1
-    s = np.asarray(scores, np.float64)
-    s = s - s.max()
-    q = np.exp(s)
-    q /= q.sum()
-    nz = p > 0
-    loss = float(np.sum(p[nz] * (np.log(p[nz]) - np.log(q[nz]))))
-    return loss, p, q - p
+def indexer_kl_row(q_t, kv_rows, scale: float, scores):
+    """(loss, target p [m], d loss / d scores [m]) for one row over its m selected rows."""
+    q, pq = _c(q_t, np.float64)
+    r, pr = _c(kv_rows, np.float64)
+    s, ps = _c(scores, np.float64)
+    H, Dk = q.shape
+    m = s.size
+    p, pp = _out(m)
+    g, pg = _out(m)
+    loss = lib().oracle_indexer_kl_row(pq, pr, m, H, Dk, float(scale), ps, pp, pg)
+    return float(loss), p, g
 
 
-# ---------------------------------------------------------------------------
-# sparse attention backward (sparse training stage)
-#   [jdon-sparse-train] jdon.com "DeepSeek-V3.2-Exp", sparse-training paragraph: the
-#   main model is trained on the sparse pattern (k = 2048 entries per query token),
-#   separately from the indexer's own loss.
-# Readings: the backward of stage 3 with respect to the query heads and the
-# selected latent rows, for an upstream gradient dO of the output; the selection
-# is piecewise constant and carries no gradient; a position selected by several
-# query rows, or twice by one row, receives the sum of its slots' gradients.
-
-def sparse_attn_backward_row(q_t: np.ndarray, kv_rows: np.ndarray, Dv: int, scale: float, dO: np.ndarray):
-    """(dq [H, Dk], dkv [m, Dk]): the gradients of sum(dO * o) for one query token,
-    o = softmax(scale * q_t . kv_rows^T) @ kv_rows[:, :Dv] per head.
-
-    With P the per-head softmax, dP = dO . v^T and D_h = sum_s P_hs dP_hs:
-    dz = P (dP - D), dq = scale dz . kv, and the row gradient is scale dz^T . q
-    (key, all Dk dims) plus P^T . dO (value, first Dv dims)."""
-    q_t = np.asarray(q_t, np.float64)
-    kv_rows = np.asarray(kv_rows, np.float64)
-    dO = np.asarray(dO, np.float64)
-    z = scale * (q_t @ kv_rows.T)                    # [H, m]
-    P = np.exp(z - z.max(axis=1, keepdims=True))
-    P /= P.sum(axis=1, keepdims=True)
-    v = kv_rows[:, :Dv]
-    dP = dO @ v.T                                    # [H, m]
-    D = np.sum(P * dP, axis=1, keepdims=True)        # [H, 1] = dO . o per head
-    dz = P * (dP - D)
-    dq = scale * (dz @ kv_rows)                      # [H, Dk]
-    dkv = scale * (dz.T @ q_t)                       # [m, Dk]  through the key
-    dkv[:, :Dv] += P.T @ dO                          # through the value
+def sparse_attn_backward_row(q_t, kv_rows, Dv: int, scale: float, dO):
+    """(dq [H, Dk], dkv [m, Dk]): gradients of sum(dO * o) for one query row."""
+    q, pq = _c(q_t, np.float64)
+    r, pr = _c(kv_rows, np.float64)
+    g, pg = _c(dO, np.float64)
+    H, Dk = q.shape
+    m = r.shape[0]
+    dq, p1 = _out((H, Dk))
+    dkv, p2 = _out((m, Dk))
+    lib().oracle_attn_backward_row(pq, pr, m, H, Dk, int(Dv), float(scale), pg, p1, p2)
     return dq, dkv
 
 
-def sparse_attn_backward_seq(q_rows: np.ndarray, kv_seq: np.ndarray, idx: np.ndarray, Dv: int, scale: float,
-                             dO: np.ndarray):
-    """Backward over the query rows of one sequence: q_rows [R, H, Dk], kv_seq
-    [L, Dk] (the sequence's latent rows by position), idx [R, k] (positions, -1 =
-    padding), dO [R, H, Dv]. Returns dq [R, H, Dk] and dkv [L, Dk], the latter
-    summed over every slot that selected each position. A row with no selected
-    position gets dq = 0."""
-    R, H, Dk = q_rows.shape
-    dq = np.zeros((R, H, Dk))
-    dkv = np.zeros((kv_seq.shape[0], Dk))
-    for r in range(R):
-        sel = np.asarray(idx[r])
-        sel = sel[sel >= 0]
-        if sel.size == 0:
-            continue
-        g_q, g_kv = sparse_attn_backward_row(q_rows[r], kv_seq[sel], Dv, scale, dO[r])
-        dq[r] = g_q
-        np.add.at(dkv, sel, g_kv)
+def sparse_attn_backward_seq(q_rows, kv_seq, idx, Dv: int, scale: float, dO):
+    """Backward over the query rows of one sequence: dq [R, H, Dk] and dkv [L, Dk]
+    summed over every slot that selected each position."""
+    q, pq = _c(q_rows, np.float64)
+    kv, pk = _c(kv_seq, np.float64)
+    ix, pi = _c(idx, np.int32)
+    g, pg = _c(dO, np.float64)
+    R, H, Dk = q.shape
+    L = kv.shape[0]
+    dq, p1 = _out((R, H, Dk))
+    dkv, p2 = _out((L, Dk))
+    lib().oracle_attn_backward_seq(pq, pk, L, pi, R, ix.shape[1], H, Dk, int(Dv), float(scale), pg, p1, p2)
     return dq, dkv

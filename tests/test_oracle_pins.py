@@ -268,6 +268,26 @@ def test_attention_permutation_invariant():
     assert np.allclose(o, o2, atol=1e-12) and np.allclose(l, l2, atol=1e-12)
 
 
+def dense_causal_mqa_online(q_t, kv_prefix, Dv, scale):
+    """Dense causal MQA for one token as a one-key-at-a-time online softmax: a
+    different algorithm from the oracle's two-pass softmax over a selection,
+    written here so that the invariant below checks the oracle against something
+    other than itself."""
+    H = q_t.shape[0]
+    m = np.full(H, -np.inf)
+    l = np.zeros(H)
+    acc = np.zeros((H, Dv))
+    for s in range(kv_prefix.shape[0]):
+        z = scale * (q_t @ kv_prefix[s])
+        m_new = np.maximum(m, z)
+        a = np.exp(m - m_new)
+        b = np.exp(z - m_new)
+        l = l * a + b
+        acc = acc * a[:, None] + b[:, None] * kv_prefix[s, :Dv][None, :]
+        m = m_new
+    return acc / l[:, None], m + np.log(l)
+
+
 def test_dsa_with_k_at_least_L_is_dense_causal_mqa():
     from sparse_long_context_04_b200.workloads import TINY, make_inputs
     from tests.case_utils import case_from_inputs
@@ -278,7 +298,7 @@ def test_dsa_with_k_at_least_L_is_dense_causal_mqa():
     for t in (0, 1, 17, 39):
         assert np.array_equal(res[t]["idx"][:t + 1], np.arange(t + 1))
         _, _, q = O.query_row(case, t)
-        o, l = O.dense_causal_mqa_online(q, kv[:t + 1], spec.Dv, spec.softmax_scale)
+        o, l = dense_causal_mqa_online(q, kv[:t + 1], spec.Dv, spec.softmax_scale)
         assert np.allclose(res[t]["o"], o, atol=1e-12) and np.allclose(res[t]["lse"], l, atol=1e-12)
 
 
