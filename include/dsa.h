@@ -135,6 +135,35 @@ dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const in
                                     const dsa_seq_layout *lay, int *idx, void *stream);
 
 /*
+ * Stages 1 and 2 fused, producer half (decode rows): the lightning indexer of
+ * dsa_indexer_scores without writing the score rows. For each row it writes the
+ * 12-bit histogram of its scores' order keys (the bins dsa_topk_from_candidates
+ * reads) and a candidate list that holds every key at or above a lower bound of
+ * the row's threshold bin, refreshed from the histogram while the row is scored.
+ * dsa_topk_from_candidates on its outputs gives exactly dsa_topk's selection over
+ * the scores dsa_indexer_scores would write; the candidates' scores are those
+ * scores, bit for bit.
+ * jdon.com "DeepSeek-V3.2-Exp": lightning-indexer paragraph (scores) and
+ * sparse-training paragraph (K = 2048 kept per query).
+ *   q_idx, q_scale, k_idx, k_scale, dt, w, H_I, d_I, lay: as for dsa_indexer_scores,
+ *            decode layouts only (lay->cu_q == NULL, T == batch), E4M3, H_I = 64, d_I = 128
+ *   k        the selection size the bound is kept for (>= 1)
+ *   hist     device uint32 [T][4096]; hist_coarse device uint32 [T][64] (the same
+ *            counts by the keys' top 6 bits); cand_count device int32 [T]. All three
+ *            are cleared and written by the call.
+ *   cand_score, cand_pos  device float32 / int32 [T][cap], cap >= the layout's cache
+ *            capacity (max_pages * page_size, or n_max), so no row can overflow; the
+ *            first cand_count[t] entries of row t are its candidates, in no order
+ * Buffers 4-byte aligned; q_idx, k_idx and w 16-byte aligned.
+ */
+dsa_status dsa_indexer_candidates(const void *q_idx, const float *q_scale,
+                                  const void *k_idx, const float *k_scale, dsa_dtype dt,
+                                  const float *w, int T, int H_I, int d_I,
+                                  const dsa_seq_layout *lay, int k, unsigned *hist,
+                                  unsigned *hist_coarse, float *cand_score, int *cand_pos,
+                                  int *cand_count, long long cap, void *stream);
+
+/*
  * Stage 3 — sparse MQA attention over the selected latent rows.
  * For row t and head h, over the selected set S_t = {idx[t*k+i] >= 0}:
  *   z_s = softmax_scale * (q[t,h,:] . kv[s,:])   (Dk dims),
@@ -297,10 +326,13 @@ typedef struct {
 size_t dsa_forward_workspace_size(const dsa_forward_args *a);
 
 /*
- * Indexer -> top-k -> attention for a->T rows. Prefill rows are processed in
- * chunks so that the score buffer stays within the workspace. The workspace is
- * caller-owned device memory of at least dsa_forward_workspace_size(a) bytes,
- * 256-byte aligned. No host synchronisation happens inside.
+ * Indexer -> top-k -> attention for a->T rows. Decode rows with the E4M3 indexer
+ * (cache capacity up to 262144 keys) take the fused path (dsa_indexer_candidates,
+ * then dsa_topk_from_candidates): the score rows are never written. Other calls
+ * write scores and run dsa_topk; prefill rows are processed in chunks so that the
+ * score buffer stays within the workspace. Both give the same selection. The
+ * workspace is caller-owned device memory of at least dsa_forward_workspace_size(a)
+ * bytes, 256-byte aligned. No host synchronisation happens inside.
  */
 dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_bytes,
                        void *stream);

@@ -169,10 +169,14 @@ dsa_status run_attn(const void *q, const void *kv, dsa_dtype dt, int T, int H, i
 // ---------------------------------------------------------------- forward plan
 constexpr size_t kScoreChunkBytes = size_t(1) << 30;  // score rows per prefill chunk
 
+constexpr long long kFusedMaxKeys = 262144;   // rows the candidate top-k's position bitmap covers
+
 struct FwdPlan {
   long long ld;
   int rows_per_chunk;
+  bool fused;  // decode + E4M3: indexer candidates and histograms, no score rows
   size_t off_scores, off_idx, off_attn, total;
+  size_t off_hist, off_hist_c, off_count, off_cscore, off_cpos;  // fused only
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -182,6 +186,7 @@ bool fwd_plan(const dsa_forward_args *a, int sms, FwdPlan *p) {
   const long long capn = a->lay.page_size ? (long long)a->lay.max_pages * a->lay.page_size : a->lay.n_max;
   if (capn < 1) return false;
   p->ld = (capn + 3) / 4 * 4;
+  p->fused = a->lay.cu_q == nullptr && a->idx_dt == DSA_E4M3 && capn <= kFusedMaxKeys;
   long long rows = (long long)(kScoreChunkBytes / (size_t)(p->ld * 4));
   if (rows < 1) rows = 1;
   if (rows > a->T) rows = a->T;
@@ -189,7 +194,17 @@ bool fwd_plan(const dsa_forward_args *a, int sms, FwdPlan *p) {
   p->rows_per_chunk = (int)(rows < 1 ? 1 : rows);
   size_t off = 0;
   p->off_scores = off;
-  off = align256(off + (size_t)p->rows_per_chunk * p->ld * 4);
+  if (p->fused) {
+    const size_t T = (size_t)a->T;
+    p->off_hist = off;
+    p->off_hist_c = off + T * 4096 * 4;
+    p->off_count = p->off_hist_c + T * 64 * 4;
+    p->off_cscore = align256(p->off_count + T * 4);
+    p->off_cpos = align256(p->off_cscore + T * (size_t)p->ld * 4);
+    off = align256(p->off_cpos + T * (size_t)p->ld * 4);
+  } else {
+    off = align256(off + (size_t)p->rows_per_chunk * p->ld * 4);
+  }
   p->off_idx = off;
   if (!a->idx_out) off = align256(off + (size_t)a->T * a->k * 4);
   p->off_attn = off;
@@ -293,6 +308,34 @@ dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const in
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
   return from_cuda(dsa::launch_topk_candidates(score, pos, count, cap, hist, T, k, L, idx, e,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_indexer_candidates(const void *q_idx, const float *q_scale, const void *k_idx, const float *k_scale,
+                                  dsa_dtype dt, const float *w, int T, int H_I, int d_I, const dsa_seq_layout *lay,
+                                  int k, unsigned *hist, unsigned *hist_coarse, float *cand_score, int *cand_pos,
+                                  int *cand_count, long long cap, void *stream) {
+  Layout L;
+  dsa_status s = check_layout(lay, T, &L);
+  if (s != DSA_OK) return s;
+  if (L.cu_q != nullptr || dt != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
+  // the score buffer check is skipped (no scores are written): pass a dummy that passes it
+  s = check_indexer(q_idx, q_scale, k_idx, k_scale, dt, w, H_I, d_I, L, reinterpret_cast<const float *>(16),
+                    (capacity(L) + 3) / 4 * 4);
+  if (s != DSA_OK) return s;
+  if (!hist || !hist_coarse || !cand_score || !cand_pos || !cand_count || k < 1) return DSA_ERR_INVALID_ARG;
+  if (cap < capacity(L)) return DSA_ERR_INVALID_ARG;
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(hist) | reinterpret_cast<uintptr_t>(hist_coarse) |
+                       reinterpret_cast<uintptr_t>(cand_score) | reinterpret_cast<uintptr_t>(cand_pos) |
+                       reinterpret_cast<uintptr_t>(cand_count);
+  if (a4 & 3u) return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  ErrCtx e;
+  int sms;
+  if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_indexer_fp8_fused(static_cast<const uint8_t *>(q_idx), q_scale,
+                                                 static_cast<const uint8_t *>(k_idx), k_scale, w, T, L, k, hist,
+                                                 hist_coarse, cand_count, cand_score, cand_pos, cap, e, sms,
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 dsa_status dsa_sparse_mqa_attn(const void *q, const void *kv, dsa_dtype dt, int T, int H, int Dk, int Dv,
@@ -430,6 +473,21 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_byt
   float *scores = reinterpret_cast<float *>(ws + p.off_scores);
   int *idx = a->idx_out ? a->idx_out : reinterpret_cast<int *>(ws + p.off_idx);
 
+  if (p.fused) {
+    unsigned *hist = reinterpret_cast<unsigned *>(ws + p.off_hist);
+    unsigned *hist_c = reinterpret_cast<unsigned *>(ws + p.off_hist_c);
+    int *count = reinterpret_cast<int *>(ws + p.off_count);
+    float *cscore = reinterpret_cast<float *>(ws + p.off_cscore);
+    int *cpos = reinterpret_cast<int *>(ws + p.off_cpos);
+    s = from_cuda(dsa::launch_indexer_fp8_fused(static_cast<const uint8_t *>(a->q_idx), a->q_scale,
+                                                static_cast<const uint8_t *>(a->k_idx), a->k_scale, a->w, a->T, L,
+                                                a->k, hist, hist_c, count, cscore, cpos, p.ld, e, sms, st));
+    if (s != DSA_OK) return s;
+    s = from_cuda(dsa::launch_topk_candidates(cscore, cpos, count, p.ld, hist, a->T, a->k, L, idx, e, st));
+    if (s != DSA_OK) return s;
+    return run_attn(a->q, a->kv, a->attn_dt, a->T, a->H, a->Dk, a->Dv, a->softmax_scale, idx, a->k, L, a->out,
+                    a->lse, ws + p.off_attn, p.total - p.off_attn, e, sms, st);
+  }
   const size_t qrow = (size_t)a->H_I * a->d_I * (a->idx_dt == DSA_E4M3 ? 1 : 4);
   for (int r0 = 0; r0 < a->T; r0 += p.rows_per_chunk) {
     const int n = (a->T - r0 < p.rows_per_chunk) ? a->T - r0 : p.rows_per_chunk;

@@ -51,7 +51,8 @@ struct Cfg {
   static constexpr int kEpiWarps = 8;
   static constexpr int kWarpsPerItem = G == 1 ? 4 : 8;  // decode: two groups of four warps alternate tiles
   static constexpr int kAccBufs = G == 1 ? 8 : 2;       // TMEM accumulators (N columns each)
-  static constexpr int kThreads = 32 * (kProdWarps + kMmaWarps + kEpiWarps);
+  static constexpr int kBoundWarp = kProdWarps + kMmaWarps + kEpiWarps;  // decode: the fused top-k's bound
+  static constexpr int kThreads = 32 * (kProdWarps + kMmaWarps + kEpiWarps + (G == 1 ? 1 : 0));
   static constexpr int kATile = kTileKeys * kDI;  // 16 KiB
   static constexpr int kBTile = N * kDI;          // 8 or 32 KiB
   static constexpr int kWBytes = G * kHI * 4;     // head weights of a query group
@@ -68,7 +69,17 @@ struct Params {
   const uint8_t *k_pool;  // paged pool base (scales live in the pages)
   const float *w;         // [T][64]
   int scales_bulk;        // key scales reach shared memory by bulk copy (else read per thread)
-  float *scores;          // [T][ld]
+  float *scores;          // [T][ld] (unless fuse)
+  // fused top-k (decode): instead of the scores, per row the histograms of the
+  // order keys' top 12 bits (fine) and top 6 bits (coarse), and the candidates
+  int fuse;
+  int k;
+  unsigned *hist;         // [T][4096], zero at launch
+  unsigned *hist_c;       // [T][64], zero at launch
+  int *cand_count;        // [T], zero at launch
+  float *cand_score;      // [T][cand_cap]
+  int *cand_pos;          // [T][cand_cap]
+  long long cand_cap;
   long long ld;
   int T;
   Layout L;
@@ -238,6 +249,69 @@ __device__ __forceinline__ int collect_batch(const Params &p, Cursor<G> &cur, lo
   return cnt;
 }
 
+// ------------------------------------------------------------------ fused top-k helpers
+// Order key of a score (the selection's rule): larger float, larger key; -0 and
+// +0 share a key; every NaN maps below -inf. Its top 12 bits are the row
+// histogram's bin, its top 6 bits the coarse bin.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// A lower bound on row t's final threshold bin (the bin of its k-th best key):
+// the highest fine bin with at least k keys at or above it in the histograms as
+// they stand. Every count only grows, and each count read is at most its final
+// value, so the bin found has at least k keys at or above it in the end too. The
+// coarse counts are read first; when the fine counts of the chosen coarse bin
+// have not caught up yet, that coarse bin's floor is returned. One warp.
+__device__ int row_bound(const Params &p, int t) {
+  const int lane = threadIdx.x & 31;
+  const unsigned *hc = p.hist_c + (long long)t * 64;
+  const unsigned *hf = p.hist + (long long)t * 4096;
+  const unsigned k = (unsigned)p.k;
+  // coarse bins from the top: lane l holds bins 63-2l and 62-2l
+  const unsigned c0 = __ldcg(hc + 63 - 2 * lane), c1 = __ldcg(hc + 62 - 2 * lane);
+  unsigned incl = c0 + c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned excl = incl - c0 - c1;
+  int cb = -1;
+  unsigned above = 0;
+  if (excl < k && excl + c0 >= k) {
+    cb = 63 - 2 * lane;
+    above = excl;
+  } else if (excl + c0 < k && excl + c0 + c1 >= k) {
+    cb = 62 - 2 * lane;
+    above = excl + c0;
+  }
+  const unsigned found = __ballot_sync(0xFFFFFFFFu, cb >= 0);
+  if (!found) return 0;  // fewer than k keys counted so far
+  const int src = __ffs(found) - 1;
+  cb = __shfl_sync(0xFFFFFFFFu, cb, src);
+  above = __shfl_sync(0xFFFFFFFFu, above, src);
+  // the 64 fine bins of coarse bin cb, from the top
+  const int f_hi = cb * 64 + 63;
+  const unsigned f0 = __ldcg(hf + f_hi - 2 * lane), f1 = __ldcg(hf + f_hi - 1 - 2 * lane);
+  unsigned fincl = f0 + f1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, fincl, o);
+    if (lane >= o) fincl += y;
+  }
+  const unsigned fex = above + fincl - f0 - f1;
+  int fb = -1;
+  if (fex < k && fex + f0 >= k) fb = f_hi - 2 * lane;
+  else if (fex + f0 < k && fex + f0 + f1 >= k) fb = f_hi - 1 - 2 * lane;
+  const unsigned ff = __ballot_sync(0xFFFFFFFFu, fb >= 0);
+  if (!ff) return cb * 64;
+  return __shfl_sync(0xFFFFFFFFu, fb, __ffs(ff) - 1);
+}
+
 // ------------------------------------------------------------------ kernel
 template <int G>
 __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
@@ -261,6 +335,9 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   __shared__ int s_seq;             // sequence holding the first item
   __shared__ long long s_fseq;      // flat index of the first item within that sequence
   __shared__ int s_b_turn;          // query-group loads issued so far (they are issued in group order)
+  __shared__ unsigned long long s_bound;  // fused top-k: (row << 32) | lower bound of that row's threshold bin
+  __shared__ int s_cur_row;               // fused top-k: the row the epilogue is scoring (-1: none yet)
+  __shared__ int s_epi_done;              // fused top-k: epilogue warps that have finished
 
   pdl_prologue();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,6 +424,9 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     }
     for (int j = 0; j < C::kMmaWarps; ++j) mbar_init(done_bar + j, 1);
     s_b_turn = 0;
+    s_bound = 0ull;
+    s_cur_row = -1;
+    s_epi_done = 0;
     fence_mbar_init();
   }
   if (warp == C::kMmaWarp0) {
@@ -505,6 +585,28 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
         }
       }
       __syncwarp();
+    } else if (G == 1 && warp == C::kBoundWarp) {
+      // ================= bound warp (fused top-k): about once a microsecond, a fresh
+      // lower bound of the current row's threshold bin from the global histograms
+      if (p.fuse) {
+        const unsigned long long t0 = globaltimer();
+        while (*reinterpret_cast<volatile int *>(&s_epi_done) < C::kEpiWarps) {
+          const int row = *reinterpret_cast<volatile int *>(&s_cur_row);
+          if (row >= 0) {
+            const int bnd = row_bound(p, row);
+            if (lane == 0)
+              *reinterpret_cast<volatile unsigned long long *>(&s_bound) =
+                  ((unsigned long long)(unsigned)row << 32) | (unsigned)bnd;
+          }
+          __syncwarp();
+          __nanosleep(1000);
+          if (error_raised(p.e)) break;
+          if (globaltimer() - t0 > p.e.limit) {  // the epilogue never finished: give up
+            if (lane == 0) raise_error(p.e, DEV_TIMEOUT, 0x440);
+            break;
+          }
+        }
+      }
     } else {
       // ================= epilogue warps
       const int ew = warp - C::kEpiWarp0;
@@ -589,7 +691,35 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
               a23 = make_float2(0.f, 0.f);
               const long long pos = cur.s.p_first + (long long)cur.i * G + gi;
               const int t = cur.row0() + gi;
-              if (gi < nrows && key_ok && s <= pos) p.scores[(long long)t * p.ld + s] = acc * qs[tt] * sk;
+              const float v = acc * qs[tt] * sk;
+              const bool valid = gi < nrows && key_ok && s <= pos;
+              if (G == 1 && p.fuse) {
+                // the row's histograms (one atomic per distinct bin of the warp's keys)
+                // and the candidates at or above the current bound, instead of the scores
+                const uint32_t bin = order_key(v) >> 20;
+                const unsigned same = __match_any_sync(0xFFFFFFFFu, valid ? bin : 0xFFFFFFFFu);
+                const unsigned same_c = __match_any_sync(0xFFFFFFFFu, valid ? (bin >> 6) : 0xFFFFFFFFu);
+                if (valid && lane == __ffs(same) - 1) atomicAdd(p.hist + (long long)t * 4096 + bin, __popc(same));
+                if (valid && lane == __ffs(same_c) - 1)
+                  atomicAdd(p.hist_c + (long long)t * 64 + (bin >> 6), __popc(same_c));
+                const unsigned long long bp = *reinterpret_cast<volatile unsigned long long *>(&s_bound);
+                const unsigned bnd = (int)(bp >> 32) == t ? (unsigned)bp : 0u;
+                const bool keep = valid && bin >= bnd;
+                const unsigned mask = __ballot_sync(0xFFFFFFFFu, keep);
+                int base = 0;
+                if (lane == 0 && mask) base = atomicAdd(p.cand_count + t, __popc(mask));
+                base = __shfl_sync(0xFFFFFFFFu, base, 0);
+                if (keep) {
+                  const long long slot = base + __popc(mask & ((1u << lane) - 1u));
+                  if (slot < p.cand_cap) {
+                    p.cand_score[(long long)t * p.cand_cap + slot] = v;
+                    p.cand_pos[(long long)t * p.cand_cap + slot] = s;
+                  }
+                }
+                if (lane == 0 && quad == 0) *reinterpret_cast<volatile int *>(&s_cur_row) = t;
+              } else if (valid) {
+                p.scores[(long long)t * p.ld + s] = v;
+              }
             }
             if (c + 1 < kCh) tmem_ld_wait(nv);
           }
@@ -604,6 +734,8 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           if (lane == 0) mbar_arrive(b_empty + slot);
         }
       }
+      __syncwarp();
+      if (lane == 0) atomicAdd(&s_epi_done, 1);  // the bound warp stops once all have finished
     }
   }
   if (error_raised(p.e)) {
@@ -681,8 +813,63 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
   p.T = T;
   p.L = L;
   p.e = e;
+  p.fuse = 0;
+  p.k = 0;
+  p.hist = nullptr;
+  p.hist_c = nullptr;
+  p.cand_count = nullptr;
+  p.cand_score = nullptr;
+  p.cand_pos = nullptr;
+  p.cand_cap = 0;
   if (L.cu_q == nullptr) return launch_g<1>(q, kI, p, num_sms, stream);
   return launch_g<4>(q, kI, p, num_sms, stream);
+}
+
+namespace {
+// Clears the fused top-k's histograms and candidate counts before the indexer
+// adds to them (chained by programmatic dependent launch like every kernel here).
+__global__ void zero_u32x3_kernel(unsigned *a, long long na, unsigned *b, long long nb, unsigned *c, long long nc) {
+  pdl_prologue();
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb + nc; i += stride) {
+    if (i < na) a[i] = 0u;
+    else if (i < na + nb) b[i - na] = 0u;
+    else c[i - na - nb] = 0u;
+  }
+}
+}  // namespace
+
+cudaError_t launch_indexer_fp8_fused(const uint8_t *q, const float *q_scale, const uint8_t *kI, const float *k_scale,
+                                     const float *w, int T, const Layout &L, int k, unsigned *hist, unsigned *hist_c,
+                                     int *cand_count, float *cand_score, int *cand_pos, long long cand_cap,
+                                     const ErrCtx &e, int num_sms, cudaStream_t stream) {
+  if (L.batch > 8192 || L.cu_q != nullptr) return cudaErrorInvalidValue;
+  const long long na = (long long)T * 4096, nb = (long long)T * 64, nc = T;
+  const int blocks = (int)min((na + nb + nc + 255) / 256, (long long)num_sms * 4);
+  cudaError_t err = launch_kernel(zero_u32x3_kernel, dim3(blocks), dim3(256), 0, stream, 0, hist, na, hist_c, nb,
+                                  reinterpret_cast<unsigned *>(cand_count), nc);
+  if (err != cudaSuccess) return err;
+  Params p;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.k_pool = kI;
+  p.w = w;
+  p.scores = nullptr;
+  p.scales_bulk = L.page_size != 0 ||
+                  ((L.n_max % 4) == 0 && (reinterpret_cast<uintptr_t>(k_scale) & 15u) == 0);
+  p.ld = 0;
+  p.T = T;
+  p.L = L;
+  p.e = e;
+  p.fuse = 1;
+  p.k = k;
+  p.hist = hist;
+  p.hist_c = hist_c;
+  p.cand_count = cand_count;
+  p.cand_score = cand_score;
+  p.cand_pos = cand_pos;
+  p.cand_cap = cand_cap;
+  return launch_g<1>(q, kI, p, num_sms, stream);
 }
 
 }  // namespace dsa

@@ -58,7 +58,7 @@ EXPORTS = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_attn_workspace_size
            "dsa_forward_workspace_size", "dsa_forward", "dsa_get_device_error", "dsa_set_wait_limit_ns",
            "dsa_status_string", "dsa_version", "dsa_sparse_mqa_attn_noalloc", "dsa_get_device_error_site",
            "dsa_cache_append", "dsa_indexer_kl", "dsa_sparse_mqa_attn_backward",
-           "dsa_sparse_mqa_attn_backward_workspace_size", "dsa_topk_from_candidates")
+           "dsa_sparse_mqa_attn_backward_workspace_size", "dsa_topk_from_candidates", "dsa_indexer_candidates")
 
 
 def lib() -> ctypes.CDLL:
@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk.argtypes = [vp, ll, i, i, ctypes.POINTER(SeqLayout), vp, vp]
         L.dsa_topk_from_candidates.argtypes = [vp, vp, vp, ll, vp, i, i, ctypes.POINTER(SeqLayout), vp, vp]
         L.dsa_topk_from_candidates.restype = i
+        L.dsa_indexer_candidates.argtypes = [vp, vp, vp, vp, i, vp, i, i, i, ctypes.POINTER(SeqLayout), i, vp, vp,
+                                             vp, vp, vp, ll, vp]
+        L.dsa_indexer_candidates.restype = i
         L.dsa_sparse_mqa_attn_workspace_size.argtypes = [i, i, i, i, i]
         L.dsa_sparse_mqa_attn_workspace_size.restype = sz
         L.dsa_sparse_mqa_attn.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, vp, i, ctypes.POINTER(SeqLayout),
@@ -166,6 +169,20 @@ def dsa_topk(scores, k, layout: Layout, idx, T=None, stream=None):
     s = lib().dsa_topk(_p(scores), int(scores.stride(0)), int(T), int(k), ctypes.byref(layout.c), _p(idx),
                        _stream(stream))
     _check(s, "dsa_topk")
+
+
+def dsa_indexer_candidates(q_idx, q_scale, k_idx, k_scale, w, layout: Layout, k, hist, hist_coarse, cand_score,
+                           cand_pos, cand_count, stream=None):
+    """Fused indexer -> top-k, producer half (decode rows): each row's 12-bit (and
+    6-bit) order-key histograms and its candidates, instead of its scores (see
+    include/dsa.h). cand_score/cand_pos [T][cap] with cap >= the cache capacity."""
+    T = int(q_idx.shape[0])
+    H_I, d_I = int(q_idx.shape[1]), int(q_idx.shape[2])
+    cap = int(cand_score.shape[1])
+    s = lib().dsa_indexer_candidates(_p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _dt(q_idx), _p(w), T, H_I, d_I,
+                                     ctypes.byref(layout.c), int(k), _p(hist), _p(hist_coarse), _p(cand_score),
+                                     _p(cand_pos), _p(cand_count), cap, _stream(stream))
+    _check(s, "dsa_indexer_candidates")
 
 
 def dsa_topk_from_candidates(score, pos, count, hist, k, layout: Layout, idx, stream=None):
