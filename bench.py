@@ -225,7 +225,6 @@ def main():
     # the fused indexer -> top-k (what dsa_forward runs on decode rows): histograms
     # and candidates instead of score rows
     hist = torch.empty((T, 4096), dtype=torch.int32, device=dev)
-    hist_c = torch.empty((T, 64), dtype=torch.int32, device=dev)
     cand_s = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
     cand_p = torch.empty((T, dc.ld), dtype=torch.int32, device=dev)
     cand_n = torch.empty((T,), dtype=torch.int32, device=dev)
@@ -237,8 +236,8 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, s.k, hist, hist_c,
-                                 cand_s, cand_p, cand_n)
+        D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, s.k, hist, cand_s,
+                                 cand_p, cand_n)
         if ev is not None:
             ev[1].record(stream)
         D.dsa_topk_from_candidates(cand_s, cand_p, cand_n, hist, s.k, dc.layout, idx)

@@ -115,15 +115,19 @@ dsa_status dsa_topk(const float *scores, long long ld, int T, int k,
  * Order key of a score x (the rule dsa_topk ranks by): 0 for NaN; otherwise, with
  * u the bits of x and -0 taken as +0, u | 0x80000000 for x >= 0 and ~u for x < 0.
  * The bin of x is its order key >> 20 (4096 bins).
- *   hist    device uint32 [T][4096]: for each row, how many of its scores
- *           s = 0..pos_t fall in each bin (all pos_t + 1 of them)
  *   score, pos  device float32 / int32 [T][cap]: each row's candidates, any order,
  *           each position at most once. Every position whose bin is at or above
  *           the row's threshold bin (the bin of its k-th best key) must be there;
  *           a producer gets this by keeping each key whose bin is at or above any
- *           lower bound of the threshold bin, e.g. one read from the row's
- *           histogram so far (the highest bin with at least k keys at or above).
+ *           lower bound of the threshold bin, e.g. one read from a histogram of
+ *           the row's keys so far (the highest bin with at least k keys at or above).
  *           Candidates below the threshold bin are ignored.
+ *   hist    device uint32 [T][4096]: per row and bin, a count that is exact for
+ *           every bin at or above the row's threshold bin (there it counts the
+ *           row's scores in the bin, all of which are candidates), with at least
+ *           min(k, pos_t + 1) in total; lower bins may hold any count. The
+ *           histogram of all the row's scores qualifies, and so does the
+ *           histogram of its candidates.
  *   count   device int32 [T]: candidates per row (<= cap)
  *   idx     device int32 [T][k], as dsa_topk writes it
  * Rows up to 262144 keys; k >= 1. A histogram or candidate list that breaks the
@@ -136,32 +140,32 @@ dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const in
 
 /*
  * Stages 1 and 2 fused, producer half (decode rows): the lightning indexer of
- * dsa_indexer_scores without writing the score rows. For each row it writes the
- * 12-bit histogram of its scores' order keys (the bins dsa_topk_from_candidates
- * reads) and a candidate list that holds every key at or above a lower bound of
- * the row's threshold bin, refreshed from the histogram while the row is scored.
- * dsa_topk_from_candidates on its outputs gives exactly dsa_topk's selection over
- * the scores dsa_indexer_scores would write; the candidates' scores are those
- * scores, bit for bit.
+ * dsa_indexer_scores without writing the score rows. For each row it writes a
+ * candidate list, which holds every key at or above a lower bound of the row's
+ * threshold bin that is refreshed from the list's own histogram while the row is
+ * scored, and that histogram (the candidates' order-key bins, as
+ * dsa_topk_from_candidates reads them). dsa_topk_from_candidates on its outputs
+ * gives exactly dsa_topk's selection over the scores dsa_indexer_scores would
+ * write; the candidates' scores are those scores, bit for bit.
  * jdon.com "DeepSeek-V3.2-Exp": lightning-indexer paragraph (scores) and
  * sparse-training paragraph (K = 2048 kept per query).
  *   q_idx, q_scale, k_idx, k_scale, dt, w, H_I, d_I, lay: as for dsa_indexer_scores,
  *            decode layouts only (lay->cu_q == NULL, T == batch), E4M3, H_I = 64, d_I = 128
  *   k        the selection size the bound is kept for (>= 1)
- *   hist     device uint32 [T][4096]; hist_coarse device uint32 [T][64] (the same
- *            counts by the keys' top 6 bits); cand_count device int32 [T]. All three
- *            are cleared and written by the call.
+ *   hist     device uint32 [T][4096], 16-byte aligned: per row, the candidates in each bin
+ *   cand_count  device int32 [T]: candidates per row. hist and cand_count are
+ *            cleared and written by the call.
  *   cand_score, cand_pos  device float32 / int32 [T][cap], cap >= the layout's cache
  *            capacity (max_pages * page_size, or n_max), so no row can overflow; the
  *            first cand_count[t] entries of row t are its candidates, in no order
- * Buffers 4-byte aligned; q_idx, k_idx and w 16-byte aligned.
+ * cand_score, cand_pos, cand_count 4-byte aligned; q_idx, k_idx and w 16-byte aligned.
  */
 dsa_status dsa_indexer_candidates(const void *q_idx, const float *q_scale,
                                   const void *k_idx, const float *k_scale, dsa_dtype dt,
                                   const float *w, int T, int H_I, int d_I,
                                   const dsa_seq_layout *lay, int k, unsigned *hist,
-                                  unsigned *hist_coarse, float *cand_score, int *cand_pos,
-                                  int *cand_count, long long cap, void *stream);
+                                  float *cand_score, int *cand_pos, int *cand_count,
+                                  long long cap, void *stream);
 
 /*
  * Stage 3 — sparse MQA attention over the selected latent rows.

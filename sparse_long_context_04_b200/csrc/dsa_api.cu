@@ -176,7 +176,7 @@ struct FwdPlan {
   int rows_per_chunk;
   bool fused;  // decode + E4M3: indexer candidates and histograms, no score rows
   size_t off_scores, off_idx, off_attn, total;
-  size_t off_hist, off_hist_c, off_count, off_cscore, off_cpos;  // fused only
+  size_t off_hist, off_count, off_cscore, off_cpos;  // fused only
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -197,8 +197,7 @@ bool fwd_plan(const dsa_forward_args *a, int sms, FwdPlan *p) {
   if (p->fused) {
     const size_t T = (size_t)a->T;
     p->off_hist = off;
-    p->off_hist_c = off + T * 4096 * 4;
-    p->off_count = p->off_hist_c + T * 64 * 4;
+    p->off_count = off + T * 4096 * 4;
     p->off_cscore = align256(p->off_count + T * 4);
     p->off_cpos = align256(p->off_cscore + T * (size_t)p->ld * 4);
     off = align256(p->off_cpos + T * (size_t)p->ld * 4);
@@ -312,8 +311,8 @@ dsa_status dsa_topk_from_candidates(const float *score, const int *pos, const in
 
 dsa_status dsa_indexer_candidates(const void *q_idx, const float *q_scale, const void *k_idx, const float *k_scale,
                                   dsa_dtype dt, const float *w, int T, int H_I, int d_I, const dsa_seq_layout *lay,
-                                  int k, unsigned *hist, unsigned *hist_coarse, float *cand_score, int *cand_pos,
-                                  int *cand_count, long long cap, void *stream) {
+                                  int k, unsigned *hist, float *cand_score, int *cand_pos, int *cand_count,
+                                  long long cap, void *stream) {
   Layout L;
   dsa_status s = check_layout(lay, T, &L);
   if (s != DSA_OK) return s;
@@ -322,19 +321,18 @@ dsa_status dsa_indexer_candidates(const void *q_idx, const float *q_scale, const
   s = check_indexer(q_idx, q_scale, k_idx, k_scale, dt, w, H_I, d_I, L, reinterpret_cast<const float *>(16),
                     (capacity(L) + 3) / 4 * 4);
   if (s != DSA_OK) return s;
-  if (!hist || !hist_coarse || !cand_score || !cand_pos || !cand_count || k < 1) return DSA_ERR_INVALID_ARG;
+  if (!hist || !cand_score || !cand_pos || !cand_count || k < 1) return DSA_ERR_INVALID_ARG;
   if (cap < capacity(L)) return DSA_ERR_INVALID_ARG;
-  const uintptr_t a4 = reinterpret_cast<uintptr_t>(hist) | reinterpret_cast<uintptr_t>(hist_coarse) |
-                       reinterpret_cast<uintptr_t>(cand_score) | reinterpret_cast<uintptr_t>(cand_pos) |
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(cand_score) | reinterpret_cast<uintptr_t>(cand_pos) |
                        reinterpret_cast<uintptr_t>(cand_count);
-  if (a4 & 3u) return DSA_ERR_INVALID_ARG;
+  if ((a4 & 3u) || !a16(hist)) return DSA_ERR_INVALID_ARG;
   if (T == 0) return DSA_OK;
   ErrCtx e;
   int sms;
   if (!device_ctx(&e, &sms)) return DSA_ERR_CUDA;
   return from_cuda(dsa::launch_indexer_fp8_fused(static_cast<const uint8_t *>(q_idx), q_scale,
                                                  static_cast<const uint8_t *>(k_idx), k_scale, w, T, L, k, hist,
-                                                 hist_coarse, cand_count, cand_score, cand_pos, cap, e, sms,
+                                                 cand_count, cand_score, cand_pos, cap, e, sms,
                                                  static_cast<cudaStream_t>(stream)));
 }
 
@@ -475,13 +473,12 @@ dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_byt
 
   if (p.fused) {
     unsigned *hist = reinterpret_cast<unsigned *>(ws + p.off_hist);
-    unsigned *hist_c = reinterpret_cast<unsigned *>(ws + p.off_hist_c);
     int *count = reinterpret_cast<int *>(ws + p.off_count);
     float *cscore = reinterpret_cast<float *>(ws + p.off_cscore);
     int *cpos = reinterpret_cast<int *>(ws + p.off_cpos);
     s = from_cuda(dsa::launch_indexer_fp8_fused(static_cast<const uint8_t *>(a->q_idx), a->q_scale,
                                                 static_cast<const uint8_t *>(a->k_idx), a->k_scale, a->w, a->T, L,
-                                                a->k, hist, hist_c, count, cscore, cpos, p.ld, e, sms, st));
+                                                a->k, hist, count, cscore, cpos, p.ld, e, sms, st));
     if (s != DSA_OK) return s;
     s = from_cuda(dsa::launch_topk_candidates(cscore, cpos, count, p.ld, hist, a->T, a->k, L, idx, e, st));
     if (s != DSA_OK) return s;

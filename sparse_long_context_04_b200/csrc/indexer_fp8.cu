@@ -70,12 +70,12 @@ struct Params {
   const float *w;         // [T][64]
   int scales_bulk;        // key scales reach shared memory by bulk copy (else read per thread)
   float *scores;          // [T][ld] (unless fuse)
-  // fused top-k (decode): instead of the scores, per row the histograms of the
-  // order keys' top 12 bits (fine) and top 6 bits (coarse), and the candidates
+  // fused top-k (decode): instead of the scores, per row the candidates (keys at
+  // or above a lower bound of the row's threshold bin) and their histogram by the
+  // top 12 bits of the order key
   int fuse;
   int k;
-  unsigned *hist;         // [T][4096], zero at launch
-  unsigned *hist_c;       // [T][64], zero at launch
+  unsigned *hist;         // [T][4096], zero at launch, 16-byte aligned
   int *cand_count;        // [T], zero at launch
   float *cand_score;      // [T][cand_cap]
   int *cand_pos;          // [T][cand_cap]
@@ -260,56 +260,52 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// A lower bound on row t's final threshold bin (the bin of its k-th best key):
-// the highest fine bin with at least k keys at or above it in the histograms as
-// they stand. Every count only grows, and each count read is at most its final
-// value, so the bin found has at least k keys at or above it in the end too. The
-// coarse counts are read first; when the fine counts of the chosen coarse bin
-// have not caught up yet, that coarse bin's floor is returned. One warp.
-__device__ int row_bound(const Params &p, int t) {
+// A lower bound on row t's final threshold bin (the bin of its k-th best key),
+// not below `cur` (the previous one): the highest bin with at least k candidates
+// at or above it in the candidates' histogram as it stands. Only bins at or above
+// the current bound are counted (keys below it are not candidates), and a later
+// bound can only be higher, so the bins below it never matter again. Each count
+// read is at most its final value and at most the row's number of scores in that
+// bin, so the bin found has at least k of the row's keys at or above it in the
+// end. One warp: a pass over bins [cur rounded down to 128, 4096), then the
+// bins of the lane where the count crosses k.
+__device__ int row_bound(const Params &p, int t, int cur) {
   const int lane = threadIdx.x & 31;
-  const unsigned *hc = p.hist_c + (long long)t * 64;
-  const unsigned *hf = p.hist + (long long)t * 4096;
   const unsigned k = (unsigned)p.k;
-  // coarse bins from the top: lane l holds bins 63-2l and 62-2l
-  const unsigned c0 = __ldcg(hc + 63 - 2 * lane), c1 = __ldcg(hc + 62 - 2 * lane);
-  unsigned incl = c0 + c1;
+  const unsigned *hf = p.hist + (long long)t * 4096;
+  const int lo = cur & ~127;
+  const int per = (4096 - lo) >> 5;  // bins per lane: a multiple of 4, 4..128
+  const int b0 = lo + lane * per;    // this lane's bins [b0, b0 + per)
+  unsigned mine = 0;
+  for (int j = 0; j < per; j += 4) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(hf + b0 + j));
+    mine += v.x + v.y + v.z + v.w;
+  }
+  unsigned suf = mine;  // candidates in this lane's bins and those of the lanes above
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += y;
+    const unsigned y = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+    if (lane + o < 32) suf += y;
   }
-  const unsigned excl = incl - c0 - c1;
-  int cb = -1;
-  unsigned above = 0;
-  if (excl < k && excl + c0 >= k) {
-    cb = 63 - 2 * lane;
-    above = excl;
-  } else if (excl + c0 < k && excl + c0 + c1 >= k) {
-    cb = 62 - 2 * lane;
-    above = excl + c0;
-  }
-  const unsigned found = __ballot_sync(0xFFFFFFFFu, cb >= 0);
-  if (!found) return 0;  // fewer than k keys counted so far
-  const int src = __ffs(found) - 1;
-  cb = __shfl_sync(0xFFFFFFFFu, cb, src);
-  above = __shfl_sync(0xFFFFFFFFu, above, src);
-  // the 64 fine bins of coarse bin cb, from the top
-  const int f_hi = cb * 64 + 63;
-  const unsigned f0 = __ldcg(hf + f_hi - 2 * lane), f1 = __ldcg(hf + f_hi - 1 - 2 * lane);
-  unsigned fincl = f0 + f1;
+  const unsigned hit = __ballot_sync(0xFFFFFFFFu, suf - mine < k && suf >= k);
+  if (!hit) return cur;  // fewer than k counted in the window so far
+  const int src = __ffs(hit) - 1;
+  const int top = __shfl_sync(0xFFFFFFFFu, b0, src) + per - 1;  // highest bin of the crossing lane
+  unsigned run = __shfl_sync(0xFFFFFFFFu, suf - mine, src);      // candidates above `top`
+  for (int c0 = 0; c0 < per; c0 += 32) {
+    const int bin = top - c0 - lane;
+    const unsigned cnt = c0 + lane < per ? __ldcg(hf + bin) : 0u;
+    unsigned incl = cnt;  // this bin and the higher ones of this chunk
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, fincl, o);
-    if (lane >= o) fincl += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned f = __ballot_sync(0xFFFFFFFFu, run + incl - cnt < k && run + incl >= k);
+    if (f) return max(cur, __shfl_sync(0xFFFFFFFFu, bin, __ffs(f) - 1));
+    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
   }
-  const unsigned fex = above + fincl - f0 - f1;
-  int fb = -1;
-  if (fex < k && fex + f0 >= k) fb = f_hi - 2 * lane;
-  else if (fex + f0 < k && fex + f0 + f1 >= k) fb = f_hi - 1 - 2 * lane;
-  const unsigned ff = __ballot_sync(0xFFFFFFFFu, fb >= 0);
-  if (!ff) return cb * 64;
-  return __shfl_sync(0xFFFFFFFFu, fb, __ffs(ff) - 1);
+  return cur;  // the lane's bins grew after the first pass; keep the bound
 }
 
 // ------------------------------------------------------------------ kernel
@@ -593,7 +589,8 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
         while (*reinterpret_cast<volatile int *>(&s_epi_done) < C::kEpiWarps) {
           const int row = *reinterpret_cast<volatile int *>(&s_cur_row);
           if (row >= 0) {
-            const int bnd = row_bound(p, row);
+            const unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(&s_bound);
+            const int bnd = row_bound(p, row, (int)(old >> 32) == row ? (int)(unsigned)old : 0);
             if (lane == 0)
               *reinterpret_cast<volatile unsigned long long *>(&s_bound) =
                   ((unsigned long long)(unsigned)row << 32) | (unsigned)bnd;
@@ -620,6 +617,23 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
       float qs[kTokPerWarp];
       for (int tt = 0; tt < kTokPerWarp; ++tt) qs[tt] = 0.f;
       bool ok = true;
+      // fused top-k: this warp's previous candidates, stored once their slot base
+      // (an atomic's return) has arrived, so that no tile waits for it
+      bool pend_keep = false;
+      unsigned pend_mask = 0u;
+      int pend_base = 0, pend_s = 0, pend_t = 0;
+      float pend_v = 0.f;
+      auto flush_pending = [&]() {
+        const int pb = __shfl_sync(0xFFFFFFFFu, pend_base, 0);
+        if (pend_keep) {
+          const long long slot = pb + __popc(pend_mask & ((1u << lane) - 1u));
+          if (slot < p.cand_cap) {
+            p.cand_score[(long long)pend_t * p.cand_cap + slot] = pend_v;
+            p.cand_pos[(long long)pend_t * p.cand_cap + slot] = pend_s;
+          }
+        }
+        pend_keep = false;
+      };
       for (long long n = 0; n < n_items; ++n) {
         const int g = cur.gcount - 1;
         const int slot = g & 1;
@@ -694,28 +708,23 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
               const float v = acc * qs[tt] * sk;
               const bool valid = gi < nrows && key_ok && s <= pos;
               if (G == 1 && p.fuse) {
-                // the row's histograms (one atomic per distinct bin of the warp's keys)
-                // and the candidates at or above the current bound, instead of the scores
+                // the candidates at or above the current bound and their histogram
+                // (fire-and-forget atomics), instead of the scores
                 const uint32_t bin = order_key(v) >> 20;
-                const unsigned same = __match_any_sync(0xFFFFFFFFu, valid ? bin : 0xFFFFFFFFu);
-                const unsigned same_c = __match_any_sync(0xFFFFFFFFu, valid ? (bin >> 6) : 0xFFFFFFFFu);
-                if (valid && lane == __ffs(same) - 1) atomicAdd(p.hist + (long long)t * 4096 + bin, __popc(same));
-                if (valid && lane == __ffs(same_c) - 1)
-                  atomicAdd(p.hist_c + (long long)t * 64 + (bin >> 6), __popc(same_c));
                 const unsigned long long bp = *reinterpret_cast<volatile unsigned long long *>(&s_bound);
                 const unsigned bnd = (int)(bp >> 32) == t ? (unsigned)bp : 0u;
                 const bool keep = valid && bin >= bnd;
+                if (keep) atomicAdd(p.hist + (long long)t * 4096 + bin, 1u);
                 const unsigned mask = __ballot_sync(0xFFFFFFFFu, keep);
+                flush_pending();
                 int base = 0;
                 if (lane == 0 && mask) base = atomicAdd(p.cand_count + t, __popc(mask));
-                base = __shfl_sync(0xFFFFFFFFu, base, 0);
-                if (keep) {
-                  const long long slot = base + __popc(mask & ((1u << lane) - 1u));
-                  if (slot < p.cand_cap) {
-                    p.cand_score[(long long)t * p.cand_cap + slot] = v;
-                    p.cand_pos[(long long)t * p.cand_cap + slot] = s;
-                  }
-                }
+                pend_base = base;
+                pend_keep = keep;
+                pend_mask = mask;
+                pend_v = v;
+                pend_s = s;
+                pend_t = t;
                 if (lane == 0 && quad == 0) *reinterpret_cast<volatile int *>(&s_cur_row) = t;
               } else if (valid) {
                 p.scores[(long long)t * p.ld + s] = v;
@@ -734,6 +743,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           if (lane == 0) mbar_arrive(b_empty + slot);
         }
       }
+      if (G == 1 && p.fuse) flush_pending();
       __syncwarp();
       if (lane == 0) atomicAdd(&s_epi_done, 1);  // the bound warp stops once all have finished
     }
@@ -816,7 +826,6 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
   p.fuse = 0;
   p.k = 0;
   p.hist = nullptr;
-  p.hist_c = nullptr;
   p.cand_count = nullptr;
   p.cand_score = nullptr;
   p.cand_pos = nullptr;
@@ -828,26 +837,25 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
 namespace {
 // Clears the fused top-k's histograms and candidate counts before the indexer
 // adds to them (chained by programmatic dependent launch like every kernel here).
-__global__ void zero_u32x3_kernel(unsigned *a, long long na, unsigned *b, long long nb, unsigned *c, long long nc) {
+__global__ void zero_u32x2_kernel(unsigned *a, long long na, unsigned *b, long long nb) {
   pdl_prologue();
   const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb + nc; i += stride) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb; i += stride) {
     if (i < na) a[i] = 0u;
-    else if (i < na + nb) b[i - na] = 0u;
-    else c[i - na - nb] = 0u;
+    else b[i - na] = 0u;
   }
 }
 }  // namespace
 
 cudaError_t launch_indexer_fp8_fused(const uint8_t *q, const float *q_scale, const uint8_t *kI, const float *k_scale,
-                                     const float *w, int T, const Layout &L, int k, unsigned *hist, unsigned *hist_c,
-                                     int *cand_count, float *cand_score, int *cand_pos, long long cand_cap,
-                                     const ErrCtx &e, int num_sms, cudaStream_t stream) {
+                                     const float *w, int T, const Layout &L, int k, unsigned *hist, int *cand_count,
+                                     float *cand_score, int *cand_pos, long long cand_cap, const ErrCtx &e,
+                                     int num_sms, cudaStream_t stream) {
   if (L.batch > 8192 || L.cu_q != nullptr) return cudaErrorInvalidValue;
-  const long long na = (long long)T * 4096, nb = (long long)T * 64, nc = T;
-  const int blocks = (int)min((na + nb + nc + 255) / 256, (long long)num_sms * 4);
-  cudaError_t err = launch_kernel(zero_u32x3_kernel, dim3(blocks), dim3(256), 0, stream, 0, hist, na, hist_c, nb,
-                                  reinterpret_cast<unsigned *>(cand_count), nc);
+  const long long na = (long long)T * 4096, nb = T;
+  const int blocks = (int)min((na + nb + 255) / 256, (long long)num_sms * 4);
+  cudaError_t err = launch_kernel(zero_u32x2_kernel, dim3(blocks), dim3(256), 0, stream, 0, hist, na,
+                                  reinterpret_cast<unsigned *>(cand_count), nb);
   if (err != cudaSuccess) return err;
   Params p;
   p.q_scale = q_scale;
@@ -864,7 +872,6 @@ cudaError_t launch_indexer_fp8_fused(const uint8_t *q, const float *q_scale, con
   p.fuse = 1;
   p.k = k;
   p.hist = hist;
-  p.hist_c = hist_c;
   p.cand_count = cand_count;
   p.cand_score = cand_score;
   p.cand_pos = cand_pos;

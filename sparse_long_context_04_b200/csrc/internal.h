@@ -58,13 +58,13 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
                                int num_sms, cudaStream_t stream);
 
 // the same indexer for decode rows with the producer half of the fused top-k: instead
-// of the scores, each row's 12-bit and 6-bit order-key histograms and the keys at or
-// above a refreshed lower bound of the row's threshold bin (hist, hist_c and
-// cand_count are cleared first, by a kernel on the same stream)
+// of the scores, the keys at or above a refreshed lower bound of each row's threshold
+// bin and their 12-bit order-key histogram (hist and cand_count are cleared first, by a
+// kernel on the same stream)
 cudaError_t launch_indexer_fp8_fused(const uint8_t *q, const float *q_scale, const uint8_t *kI, const float *k_scale,
-                                     const float *w, int T, const Layout &L, int k, unsigned *hist, unsigned *hist_c,
-                                     int *cand_count, float *cand_score, int *cand_pos, long long cand_cap,
-                                     const ErrCtx &e, int num_sms, cudaStream_t stream);
+                                     const float *w, int T, const Layout &L, int k, unsigned *hist, int *cand_count,
+                                     float *cand_score, int *cand_pos, long long cand_cap, const ErrCtx &e,
+                                     int num_sms, cudaStream_t stream);
 
 // bf16 tcgen05 sparse MQA attention (attn_bf16.cu): H = 128, Dk = 576, Dv = 512
 struct AttnPlan {

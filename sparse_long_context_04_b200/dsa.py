@@ -74,7 +74,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk_from_candidates.argtypes = [vp, vp, vp, ll, vp, i, i, ctypes.POINTER(SeqLayout), vp, vp]
         L.dsa_topk_from_candidates.restype = i
         L.dsa_indexer_candidates.argtypes = [vp, vp, vp, vp, i, vp, i, i, i, ctypes.POINTER(SeqLayout), i, vp, vp,
-                                             vp, vp, vp, ll, vp]
+                                             vp, vp, ll, vp]
         L.dsa_indexer_candidates.restype = i
         L.dsa_sparse_mqa_attn_workspace_size.argtypes = [i, i, i, i, i]
         L.dsa_sparse_mqa_attn_workspace_size.restype = sz
@@ -171,17 +171,17 @@ def dsa_topk(scores, k, layout: Layout, idx, T=None, stream=None):
     _check(s, "dsa_topk")
 
 
-def dsa_indexer_candidates(q_idx, q_scale, k_idx, k_scale, w, layout: Layout, k, hist, hist_coarse, cand_score,
-                           cand_pos, cand_count, stream=None):
-    """Fused indexer -> top-k, producer half (decode rows): each row's 12-bit (and
-    6-bit) order-key histograms and its candidates, instead of its scores (see
+def dsa_indexer_candidates(q_idx, q_scale, k_idx, k_scale, w, layout: Layout, k, hist, cand_score, cand_pos,
+                           cand_count, stream=None):
+    """Fused indexer -> top-k, producer half (decode rows): each row's candidates
+    and their 12-bit order-key histogram, instead of its scores (see
     include/dsa.h). cand_score/cand_pos [T][cap] with cap >= the cache capacity."""
     T = int(q_idx.shape[0])
     H_I, d_I = int(q_idx.shape[1]), int(q_idx.shape[2])
     cap = int(cand_score.shape[1])
     s = lib().dsa_indexer_candidates(_p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _dt(q_idx), _p(w), T, H_I, d_I,
-                                     ctypes.byref(layout.c), int(k), _p(hist), _p(hist_coarse), _p(cand_score),
-                                     _p(cand_pos), _p(cand_count), cap, _stream(stream))
+                                     ctypes.byref(layout.c), int(k), _p(hist), _p(cand_score), _p(cand_pos),
+                                     _p(cand_count), cap, _stream(stream))
     _check(s, "dsa_indexer_candidates")
 
 

@@ -5,10 +5,10 @@ decode rows.
 
 Checked against the GPU's own unfused scores (dsa_indexer_scores, the same
 indexer arithmetic):
-  - each row's 12-bit and 6-bit histograms equal the histograms of its scores;
   - every candidate's score equals the unfused score at its position, bit for
     bit; positions are distinct and causal; every key at or above the row's
-    threshold bin is a candidate;
+    threshold bin is a candidate; each row's 12-bit histogram counts exactly its
+    candidates;
   - dsa_forward's selection equals the oracle's top-k of the unfused scores on
     every row, and its attention output equals the attention on that selection;
   - on rows built to defeat the filter: equal scores everywhere (one bin holds
@@ -32,33 +32,30 @@ def _producer(dc, k):
     T, cap = dc.T, dc.ld
     dev = dc.q.device
     hist = torch.full((T, 4096), 7, dtype=torch.int32, device=dev)     # not zero: the call clears it
-    hist_c = torch.full((T, 64), 7, dtype=torch.int32, device=dev)
     cs = torch.empty((T, cap), dtype=torch.float32, device=dev)
     cp = torch.empty((T, cap), dtype=torch.int32, device=dev)
     cnt = torch.full((T,), 7, dtype=torch.int32, device=dev)
-    D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, k, hist, hist_c, cs, cp,
-                             cnt)
+    D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, k, hist, cs, cp, cnt)
     torch.cuda.synchronize()
     assert D.dsa_get_device_error_site() == (D.DSA_OK, 0)
-    return hist.cpu().numpy(), hist_c.cpu().numpy(), cs.cpu().numpy(), cp.cpu().numpy(), cnt.cpu().numpy()
+    return hist.cpu().numpy(), cs.cpu().numpy(), cp.cpu().numpy(), cnt.cpu().numpy()
 
 
 def _check(dc, k):
     pos = dc.inp.pos.numpy()
     scores = G.indexer(dc).cpu().numpy()
-    hist, hist_c, cs, cp, cnt = _producer(dc, k)
+    hist, cs, cp, cnt = _producer(dc, k)
     kept = 0
     for t in range(dc.T):
         n = int(pos[t]) + 1
         row = scores[t, :n]
         bins = (order_key(row) >> 20).astype(np.int64)
-        assert np.array_equal(hist[t], np.bincount(bins, minlength=4096)), t
-        assert np.array_equal(hist_c[t], np.bincount(bins >> 6, minlength=64)), t
         c = int(cnt[t])
         assert 0 < c <= dc.ld, (t, c)
         p = cp[t, :c]
         assert np.unique(p).size == c and p.min() >= 0 and p.max() < n, t
         assert np.array_equal(cs[t, :c].view(np.uint32), row[p].view(np.uint32)), t
+        assert np.array_equal(hist[t], np.bincount(bins[p], minlength=4096)), t   # the candidates' histogram
         sel = O.topk_row(row, k)
         sel = sel[sel >= 0]
         thr_bin = int((order_key(row[sel]) >> 20).min())

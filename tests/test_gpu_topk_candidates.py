@@ -1,7 +1,8 @@
 """Top-k from a filtered candidate list (dsa_topk_from_candidates) against the
 oracle's top-k over the full row.
 
-The candidates and the 12-bit histograms are built on the host the way a fused
+The candidates and the 12-bit histograms (of the whole row, or of the candidates
+only, as the fused indexer hands them over) are built on the host the way a fused
 indexer keeps them: keys arrive tile by tile, each tile is filtered against a
 lower bound of the row's threshold bin read from the histogram so far (stale by
 a random number of tiles), and the survivors are stored in a shuffled order.
@@ -37,7 +38,7 @@ def _candidates(x, k, rng, tile=128):
     return hist.astype(np.uint32), keep
 
 
-def _run(rows, k, seed=0, corrupt_row=None):
+def _run(rows, k, seed=0, corrupt_row=None, hist_of="all"):
     ensure_lib()
     rng = np.random.default_rng(seed)
     T = len(rows)
@@ -49,6 +50,8 @@ def _run(rows, k, seed=0, corrupt_row=None):
     hist = np.zeros((T, 4096), np.uint32)
     for t, x in enumerate(rows):
         h, keep = _candidates(x, k, rng)
+        if hist_of == "candidates":   # the fused indexer hands over the candidates' histogram
+            h = np.bincount((order_key(x[keep]) >> 20).astype(np.int64), minlength=4096).astype(np.uint32)
         hist[t] = h
         count[t] = keep.size
         score[t, :keep.size] = x[keep]
@@ -89,11 +92,12 @@ def _rows(rng, T):
     return out
 
 
+@pytest.mark.parametrize("hist_of", ["all", "candidates"])
 @pytest.mark.parametrize("k", [1, 64, 2048])
-def test_topk_from_candidates_equals_full_topk(k):
+def test_topk_from_candidates_equals_full_topk(k, hist_of):
     rng = np.random.default_rng(k)
     rows = _rows(rng, 14)
-    got = _run(rows, k, seed=k)
+    got = _run(rows, k, seed=k, hist_of=hist_of)
     assert D.dsa_get_device_error() == D.DSA_OK
     for t, x in enumerate(rows):
         assert np.array_equal(got[t], O.topk_row(x, k)), (t, x.size)
