@@ -177,38 +177,50 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   const int lane = tid & 31;
   const unsigned lt = (1u << lane) - 1u;
   // every lane of a warp runs the same iterations, so the counters take one
-  // shared-memory atomic per warp (ballot and population count), not one per key
-  for (long long i0 = tid - lane; i0 < cnt; i0 += kThreads) {
-    const long long i = i0 + lane;
-    bool is_above = false, is_tie = false;
-    uint32_t key = 0;
-    int s = 0;
-    if (i < cnt) {
-      key = order_key(__ldg(cs + i));
-      s = __ldg(cp + i);
-      const int bin = (int)(key >> 20);
-      if (bin >= B) {
-        if (s < 0 || (long long)s >= n) {
-          raise_error(p.e, DEV_BOUNDS, 0x903);
-        } else {
-          is_above = bin > B;
-          is_tie = bin == B;
+  // shared-memory atomic per warp (ballot and population count), not one per key;
+  // each lane loads kU candidates before it looks at any, so that the loads'
+  // latencies overlap
+  constexpr int kU = 8;
+  for (long long i0 = (long long)(tid - lane) * kU; i0 < cnt; i0 += (long long)kThreads * kU) {
+    float sc[kU];
+    int ps[kU];
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+      const long long i = i0 + j * 32 + lane;
+      sc[j] = i < cnt ? __ldg(cs + i) : 0.f;
+      ps[j] = i < cnt ? __ldg(cp + i) : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+      const long long i = i0 + j * 32 + lane;
+      bool is_above = false, is_tie = false;
+      const uint32_t key = order_key(sc[j]);
+      const int s = ps[j];
+      if (i < cnt) {
+        const int bin = (int)(key >> 20);
+        if (bin >= B) {
+          if (s < 0 || (long long)s >= n) {
+            raise_error(p.e, DEV_BOUNDS, 0x903);
+          } else {
+            is_above = bin > B;
+            is_tie = bin == B;
+          }
         }
       }
-    }
-    if (is_above) atomicOr(&sm.bitmap[s >> 5], 1u << (s & 31));
-    const unsigned ma = __ballot_sync(0xFFFFFFFFu, is_above), mt = __ballot_sync(0xFFFFFFFFu, is_tie);
-    unsigned tb = 0;
-    if (lane == 0) {
-      if (ma) atomicAdd(&sm.n_above, (unsigned)__popc(ma));
-      if (mt) tb = atomicAdd(&sm.n_tie, (unsigned)__popc(mt));
-    }
-    tb = __shfl_sync(0xFFFFFFFFu, tb, 0);
-    if (is_tie) {
-      const unsigned slot = tb + __popc(mt & lt);
-      if (slot < kTieCap) {
-        sm.tie_key[slot] = key;
-        sm.tie_pos[slot] = s;
+      if (is_above) atomicOr(&sm.bitmap[s >> 5], 1u << (s & 31));
+      const unsigned ma = __ballot_sync(0xFFFFFFFFu, is_above), mt = __ballot_sync(0xFFFFFFFFu, is_tie);
+      unsigned tb = 0;
+      if (lane == 0) {
+        if (ma) atomicAdd(&sm.n_above, (unsigned)__popc(ma));
+        if (mt) tb = atomicAdd(&sm.n_tie, (unsigned)__popc(mt));
+      }
+      tb = __shfl_sync(0xFFFFFFFFu, tb, 0);
+      if (is_tie) {
+        const unsigned slot = tb + __popc(mt & lt);
+        if (slot < kTieCap) {
+          sm.tie_key[slot] = key;
+          sm.tie_pos[slot] = s;
+        }
       }
     }
   }
