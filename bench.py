@@ -222,43 +222,43 @@ def main():
     lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
     wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
     ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
-    # the fused indexer -> top-k (what dsa_forward runs on decode rows): histograms
-    # and candidates instead of score rows
+    # the fused indexer -> top-k (dsa_indexer_candidates + dsa_topk_from_candidates),
+    # timed beside the step for comparison: candidates and their histogram instead
+    # of score rows
     hist = torch.empty((T, 4096), dtype=torch.int32, device=dev)
     cand_s = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
     cand_p = torch.empty((T, dc.ld), dtype=torch.int32, device=dev)
     cand_n = torch.empty((T,), dtype=torch.int32, device=dev)
-    # clear + fused indexer, candidate top-k, then attention: a kernel and a
-    # split-merge kernel per chunk of 296 rows
-    launches_per_step = 3 + 2 * ((T + 295) // 296)
+    # indexer, top-k, then attention: a kernel and a split-merge kernel per chunk of 296 rows
+    launches_per_step = 2 + 2 * ((T + 295) // 296)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, s.k, hist, cand_s,
-                                 cand_p, cand_n)
+        D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, scores)
         if ev is not None:
             ev[1].record(stream)
-        D.dsa_topk_from_candidates(cand_s, cand_p, cand_n, hist, s.k, dc.layout, idx)
+        D.dsa_topk(scores, s.k, dc.layout, idx)
         if ev is not None:
             ev[2].record(stream)
         D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws)
         if ev is not None:
             ev[3].record(stream)
 
-    def unfused_stages(reps=40):
-        """The unfused pair (score rows written, then the cluster top-k) for comparison."""
-        evs_u = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
-        for e3 in evs_u:
+    def fused_stages(reps=40):
+        """The fused pair's two stages, CUDA events around each."""
+        evs_f = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        for e3 in evs_f:
             e3[0].record(stream)
-            D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, scores)
+            D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, s.k, hist, cand_s,
+                                     cand_p, cand_n)
             e3[1].record(stream)
-            D.dsa_topk(scores, s.k, dc.layout, idx)
+            D.dsa_topk_from_candidates(cand_s, cand_p, cand_n, hist, s.k, dc.layout, idx)
             e3[2].record(stream)
         torch.cuda.synchronize(dev)
-        return {"indexer": sum(e3[0].elapsed_time(e3[1]) for e3 in evs_u) / reps * 1e3,
-                "topk": sum(e3[1].elapsed_time(e3[2]) for e3 in evs_u) / reps * 1e3}
+        return {"indexer": sum(e3[0].elapsed_time(e3[1]) for e3 in evs_f) / reps * 1e3,
+                "topk": sum(e3[1].elapsed_time(e3[2]) for e3 in evs_f) / reps * 1e3}
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -290,10 +290,12 @@ def main():
     ms = X.max_over_ranks(ms, dev)
     if D.dsa_get_device_error() != D.DSA_OK:
         raise RuntimeError("device error during timing")
+    fused = fused_stages()
     kept = int(cand_n.sum())
-    unfused = unfused_stages()   # also leaves the score rows that the indexer loss below reads
+    step()                       # the score rows and selection the indexer loss below reads
+    torch.cuda.synchronize(dev)
     if D.dsa_get_device_error() != D.DSA_OK:
-        raise RuntimeError("device error in the unfused stages")
+        raise RuntimeError("device error in the fused stages")
 
     # ---- end to end through dsa_forward with host buffers. Two slots of per-step
     # device inputs and outputs: step i+1's inputs cross PCIe (own stream) while
@@ -459,7 +461,7 @@ def main():
         return
 
     hbm, hbm_src = peaks()
-    ab = algorithmic_bytes(inp)
+    ab = algorithmic_bytes(inp, fused=False)
     step_s = ms / 1e3 / args.steps
     idx_s = stage_ms[0] / 1e3
     idx_gbs = ab["indexer"] / idx_s / 1e9
@@ -489,13 +491,13 @@ def main():
         },
         "stages_us": {"indexer": stage_ms[0] * 1e3, "topk": stage_ms[1] * 1e3, "attention": stage_ms[2] * 1e3,
                       "probed_steps": len(probed),
-                      "path": "fused indexer -> top-k (dsa_indexer_candidates + dsa_topk_from_candidates)"},
-        "fused_topk": {"candidates_kept": kept, "keys": int(inp.seq_lens.sum()),
+                      "path": "score rows (dsa_indexer_scores) + cluster top-k (dsa_topk), as dsa_forward's default"},
+        "fused_topk": {"stages_us": fused, "candidates_kept": kept, "keys": int(inp.seq_lens.sum()),
                        "kept_frac": kept / int(inp.seq_lens.sum()),
-                       "unfused_us": unfused,
-                       "note": "unfused = dsa_indexer_scores writing score rows + dsa_topk, 40 steps, for comparison"},
+                       "note": "dsa_indexer_candidates + dsa_topk_from_candidates (no score rows), 40 steps "
+                               "with events around each stage, same selection as the step's"},
         "roofline": {
-            "bound": "hbm", "kernel": "indexer_fp8_kernel (decode, N=64, fused top-k producer)",
+            "bound": "hbm", "kernel": "indexer_fp8_kernel (decode, N=64)",
             "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
             "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured" else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": ab["indexer"],

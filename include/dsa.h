@@ -324,19 +324,27 @@ typedef struct {
   /* outputs */
   void *out; float *lse;          /* lse may be NULL */
   int *idx_out;                   /* optional device int32 [T][k] copy of the selection */
+  int topk_path;                  /* how stages 1 and 2 run: DSA_TOPK_AUTO (0, the library's
+                                     choice), DSA_TOPK_SCORES (score rows, then dsa_topk) or
+                                     DSA_TOPK_FUSED (dsa_indexer_candidates, then
+                                     dsa_topk_from_candidates; decode rows with the E4M3 indexer
+                                     and a cache capacity up to 262144 keys, else as AUTO) */
 } dsa_forward_args;
+
+enum { DSA_TOPK_AUTO = 0, DSA_TOPK_SCORES = 1, DSA_TOPK_FUSED = 2 };
 
 /* Workspace bytes dsa_forward needs for these arguments (0 on invalid arguments). */
 size_t dsa_forward_workspace_size(const dsa_forward_args *a);
 
 /*
- * Indexer -> top-k -> attention for a->T rows. Decode rows with the E4M3 indexer
- * (cache capacity up to 262144 keys) take the fused path (dsa_indexer_candidates,
- * then dsa_topk_from_candidates): the score rows are never written. Other calls
- * write scores and run dsa_topk; prefill rows are processed in chunks so that the
- * score buffer stays within the workspace. Both give the same selection. The
- * workspace is caller-owned device memory of at least dsa_forward_workspace_size(a)
- * bytes, 256-byte aligned. No host synchronisation happens inside.
+ * Indexer -> top-k -> attention for a->T rows. a->topk_path picks how the selection
+ * is made: score rows then dsa_topk (prefill rows in chunks, so that the score
+ * buffer stays within the workspace), or, for decode rows, the fused pair
+ * dsa_indexer_candidates + dsa_topk_from_candidates, which writes no score rows.
+ * Both give the same selection; DSA_TOPK_AUTO takes the one measured faster on
+ * B200 for the shape (today the score rows). The workspace is caller-owned device
+ * memory of at least dsa_forward_workspace_size(a) bytes (computed for the same
+ * topk_path), 256-byte aligned. No host synchronisation happens inside.
  */
 dsa_status dsa_forward(const dsa_forward_args *a, void *workspace, size_t ws_bytes,
                        void *stream);

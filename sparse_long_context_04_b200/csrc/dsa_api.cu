@@ -182,11 +182,14 @@ struct FwdPlan {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool fwd_plan(const dsa_forward_args *a, int sms, FwdPlan *p) {
-  if (!a || a->T < 0) return false;
+  if (!a || a->T < 0 || a->topk_path < DSA_TOPK_AUTO || a->topk_path > DSA_TOPK_FUSED) return false;
   const long long capn = a->lay.page_size ? (long long)a->lay.max_pages * a->lay.page_size : a->lay.n_max;
   if (capn < 1) return false;
   p->ld = (capn + 3) / 4 * 4;
-  p->fused = a->lay.cu_q == nullptr && a->idx_dt == DSA_E4M3 && capn <= kFusedMaxKeys;
+  // the fused pair is exact on every decode shape it takes; it is not yet the faster
+  // one on B200, so only an explicit request selects it
+  p->fused = a->topk_path == DSA_TOPK_FUSED && a->lay.cu_q == nullptr && a->idx_dt == DSA_E4M3 &&
+             capn <= kFusedMaxKeys;
   long long rows = (long long)(kScoreChunkBytes / (size_t)(p->ld * 4));
   if (rows < 1) rows = 1;
   if (rows > a->T) rows = a->T;

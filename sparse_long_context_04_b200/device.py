@@ -92,7 +92,7 @@ def indexer_kl(dc: DeviceCase, idx: torch.Tensor, lse: torch.Tensor, scores: tor
 class Forward:
     """dsa_forward with its buffers allocated once (reusable across steps)."""
 
-    def __init__(self, dc: DeviceCase, keep_idx: bool = True):
+    def __init__(self, dc: DeviceCase, keep_idx: bool = True, topk_path: int = D.DSA_TOPK_AUTO):
         s = dc.inp.spec
         dev = dc.q.device
         self.dc = dc
@@ -100,7 +100,7 @@ class Forward:
         self.lse = torch.empty((dc.T, s.H), dtype=torch.float32, device=dev)
         self.idx = torch.empty((dc.T, s.k), dtype=torch.int32, device=dev) if keep_idx else None
         self.args = D.forward_args(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.q, dc.kv, s.k,
-                                   s.softmax_scale, dc.layout, self.out, self.lse, self.idx)
+                                   s.softmax_scale, dc.layout, self.out, self.lse, self.idx, topk_path)
         n = D.dsa_forward_workspace_size(self.args)
         if n == 0:
             raise D.DSAError(D.DSA_ERR_INVALID_ARG, "dsa_forward_workspace_size")

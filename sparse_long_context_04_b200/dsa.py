@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_WORKSPACE, \
     DSA_ERR_DEVICE_CHECK, DSA_ERR_TOO_LARGE = range(8)
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
+DSA_TOPK_AUTO, DSA_TOPK_SCORES, DSA_TOPK_FUSED = 0, 1, 2
 
 
 class DSAError(RuntimeError):
@@ -49,6 +50,7 @@ class ForwardArgs(ctypes.Structure):
         ("k", ctypes.c_int), ("T", ctypes.c_int),
         ("lay", SeqLayout),
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
+        ("topk_path", ctypes.c_int),
     ]
 
 
@@ -258,7 +260,7 @@ def dsa_sparse_mqa_attn_noalloc(q, kv, idx, layout: Layout, out, lse, softmax_sc
 
 
 def forward_args(q_idx, q_scale, k_idx, k_scale, w, q, kv, k, softmax_scale, layout: Layout, out, lse=None,
-                 idx_out=None) -> ForwardArgs:
+                 idx_out=None, topk_path=DSA_TOPK_AUTO) -> ForwardArgs:
     a = ForwardArgs()
     a.q_idx, a.q_scale, a.k_idx, a.k_scale = (t.data_ptr() if t is not None else None
                                               for t in (q_idx, q_scale, k_idx, k_scale))
@@ -276,6 +278,7 @@ def forward_args(q_idx, q_scale, k_idx, k_scale, w, q, kv, k, softmax_scale, lay
     a.out = out.data_ptr()
     a.lse = None if lse is None else lse.data_ptr()
     a.idx_out = None if idx_out is None else idx_out.data_ptr()
+    a.topk_path = int(topk_path)
     return a
 
 

@@ -1,7 +1,7 @@
 """The fused indexer -> top-k on decode rows: dsa_indexer_candidates (the indexer
 writing each row's order-key histograms and a filtered candidate list instead of
 its scores), dsa_topk_from_candidates, and dsa_forward, which chains them for
-decode rows.
+decode rows when asked to (topk_path = DSA_TOPK_FUSED).
 
 Checked against the GPU's own unfused scores (dsa_indexer_scores, the same
 indexer arithmetic):
@@ -68,7 +68,7 @@ def _check(dc, k):
 def _forward_check(dc, scores):
     s = dc.inp.spec
     pos = dc.inp.pos.numpy()
-    out, lse, idx = G.Forward(dc)()
+    out, lse, idx = G.Forward(dc, topk_path=D.DSA_TOPK_FUSED)()
     torch.cuda.synchronize()
     assert D.dsa_get_device_error_site() == (D.DSA_OK, 0)
     ix = idx.cpu().numpy()
