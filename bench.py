@@ -246,6 +246,25 @@ def main():
         if ev is not None:
             ev[3].record(stream)
 
+    def fused_step():
+        D.dsa_indexer_candidates(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, s.k, hist, cand_s,
+                                 cand_p, cand_n)
+        D.dsa_topk_from_candidates(cand_s, cand_p, cand_n, hist, s.k, dc.layout, idx)
+        D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws)
+
+    def fused_steps(n=200):
+        """Whole steps on the fused pair, back to back like the timed ones (ms per step)."""
+        for _ in range(5):
+            fused_step()
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n):
+            fused_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        return f0.elapsed_time(f1) / n
+
     def fused_stages(reps=40):
         """The fused pair's two stages, CUDA events around each."""
         evs_f = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
@@ -292,6 +311,7 @@ def main():
         raise RuntimeError("device error during timing")
     fused = fused_stages()
     kept = int(cand_n.sum())
+    fused_ms = fused_steps()
     step()                       # the score rows and selection the indexer loss below reads
     torch.cuda.synchronize(dev)
     if D.dsa_get_device_error() != D.DSA_OK:
@@ -492,10 +512,12 @@ def main():
         "stages_us": {"indexer": stage_ms[0] * 1e3, "topk": stage_ms[1] * 1e3, "attention": stage_ms[2] * 1e3,
                       "probed_steps": len(probed),
                       "path": "score rows (dsa_indexer_scores) + cluster top-k (dsa_topk), as dsa_forward's default"},
-        "fused_topk": {"stages_us": fused, "candidates_kept": kept, "keys": int(inp.seq_lens.sum()),
+        "fused_topk": {"ms_per_step": fused_ms, "tokens_per_s": T / (fused_ms / 1e3),
+                       "stages_us": fused, "candidates_kept": kept, "keys": int(inp.seq_lens.sum()),
                        "kept_frac": kept / int(inp.seq_lens.sum()),
-                       "note": "dsa_indexer_candidates + dsa_topk_from_candidates (no score rows), 40 steps "
-                               "with events around each stage, same selection as the step's"},
+                       "note": "dsa_indexer_candidates + dsa_topk_from_candidates (no score rows) + attention: "
+                               "200 whole steps back to back; stage times from 40 more with events around each "
+                               "stage; same selection as the step's"},
         "roofline": {
             "bound": "hbm", "kernel": "indexer_fp8_kernel (decode, N=64)",
             "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,

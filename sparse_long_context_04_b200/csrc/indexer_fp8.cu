@@ -267,14 +267,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // bound can only be higher, so the bins below it never matter again. Each count
 // read is at most its final value and at most the row's number of scores in that
 // bin, so the bin found has at least k of the row's keys at or above it in the
-// end. One warp: a pass over bins [cur rounded down to 128, 4096), then the
-// bins of the lane where the count crosses k.
-__device__ int row_bound(const Params &p, int t, int cur) {
+// end. Bins above `top` (the highest candidate bin this CTA has seen in the row)
+// are not read: leaving counts out only lowers the bound. One warp: a pass over
+// bins [cur rounded down to 128, top rounded up), then the bins of the lane where
+// the count crosses k.
+__device__ int row_bound(const Params &p, int t, int cur, int top) {
   const int lane = threadIdx.x & 31;
   const unsigned k = (unsigned)p.k;
   const unsigned *hf = p.hist + (long long)t * 4096;
   const int lo = cur & ~127;
-  const int per = (4096 - lo) >> 5;  // bins per lane: a multiple of 4, 4..128
+  const int nb = min(4096 - lo, (max(top + 1 - lo, 1) + 127) & ~127);  // a multiple of 128
+  const int per = nb >> 5;  // bins per lane: a multiple of 4, 4..128
   const int b0 = lo + lane * per;    // this lane's bins [b0, b0 + per)
   unsigned mine = 0;
   for (int j = 0; j < per; j += 4) {
@@ -290,10 +293,10 @@ __device__ int row_bound(const Params &p, int t, int cur) {
   const unsigned hit = __ballot_sync(0xFFFFFFFFu, suf - mine < k && suf >= k);
   if (!hit) return cur;  // fewer than k counted in the window so far
   const int src = __ffs(hit) - 1;
-  const int top = __shfl_sync(0xFFFFFFFFu, b0, src) + per - 1;  // highest bin of the crossing lane
-  unsigned run = __shfl_sync(0xFFFFFFFFu, suf - mine, src);      // candidates above `top`
+  const int hi = __shfl_sync(0xFFFFFFFFu, b0, src) + per - 1;  // highest bin of the crossing lane
+  unsigned run = __shfl_sync(0xFFFFFFFFu, suf - mine, src);     // candidates above `hi`
   for (int c0 = 0; c0 < per; c0 += 32) {
-    const int bin = top - c0 - lane;
+    const int bin = hi - c0 - lane;
     const unsigned cnt = c0 + lane < per ? __ldcg(hf + bin) : 0u;
     unsigned incl = cnt;  // this bin and the higher ones of this chunk
 #pragma unroll
@@ -332,7 +335,9 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   __shared__ long long s_fseq;      // flat index of the first item within that sequence
   __shared__ int s_b_turn;          // query-group loads issued so far (they are issued in group order)
   __shared__ unsigned long long s_bound;  // fused top-k: (row << 32) | lower bound of that row's threshold bin
+  __shared__ unsigned long long s_top;    // fused top-k: (row << 32) | highest candidate bin seen in that row
   __shared__ int s_cur_row;               // fused top-k: the row the epilogue is scoring (-1: none yet)
+  __shared__ int s_tiles;                 // fused top-k: tiles the epilogue has finished
   __shared__ int s_epi_done;              // fused top-k: epilogue warps that have finished
 
   pdl_prologue();
@@ -421,7 +426,9 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     for (int j = 0; j < C::kMmaWarps; ++j) mbar_init(done_bar + j, 1);
     s_b_turn = 0;
     s_bound = 0ull;
+    s_top = 0ull;
     s_cur_row = -1;
+    s_tiles = 0;
     s_epi_done = 0;
     fence_mbar_init();
   }
@@ -586,11 +593,16 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
       // lower bound of the current row's threshold bin from the global histograms
       if (p.fuse) {
         const unsigned long long t0 = globaltimer();
+        int seen = -1;  // tiles finished at the last refresh: refresh only after new ones
         while (*reinterpret_cast<volatile int *>(&s_epi_done) < C::kEpiWarps) {
           const int row = *reinterpret_cast<volatile int *>(&s_cur_row);
-          if (row >= 0) {
+          const int tiles = *reinterpret_cast<volatile int *>(&s_tiles);
+          if (row >= 0 && tiles != seen) {
+            seen = tiles;
             const unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(&s_bound);
-            const int bnd = row_bound(p, row, (int)(old >> 32) == row ? (int)(unsigned)old : 0);
+            const unsigned long long tp = *reinterpret_cast<volatile unsigned long long *>(&s_top);
+            const int bnd = row_bound(p, row, (int)(old >> 32) == row ? (int)(unsigned)old : 0,
+                                      (int)(tp >> 32) == row ? (int)(unsigned)tp : 4095);
             if (lane == 0)
               *reinterpret_cast<volatile unsigned long long *>(&s_bound) =
                   ((unsigned long long)(unsigned)row << 32) | (unsigned)bnd;
@@ -716,6 +728,9 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
                 const bool keep = valid && bin >= bnd;
                 if (keep) atomicAdd(p.hist + (long long)t * 4096 + bin, 1u);
                 const unsigned mask = __ballot_sync(0xFFFFFFFFu, keep);
+                const unsigned wtop = __reduce_max_sync(0xFFFFFFFFu, keep ? bin : 0u);
+                if (lane == 0 && mask)  // rows only increase within a CTA: (row, bin) pairs order by max
+                  atomicMax(&s_top, ((unsigned long long)(unsigned)t << 32) | wtop);
                 flush_pending();
                 int base = 0;
                 if (lane == 0 && mask) base = atomicAdd(p.cand_count + t, __popc(mask));
@@ -725,7 +740,10 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
                 pend_v = v;
                 pend_s = s;
                 pend_t = t;
-                if (lane == 0 && quad == 0) *reinterpret_cast<volatile int *>(&s_cur_row) = t;
+                if (lane == 0 && quad == 0) {
+                  *reinterpret_cast<volatile int *>(&s_cur_row) = t;
+                  atomicAdd(&s_tiles, 1);
+                }
               } else if (valid) {
                 p.scores[(long long)t * p.ld + s] = v;
               }

@@ -28,7 +28,7 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;                   // top 12 bits of the order key
 constexpr int kBinsPerThread = kBins / kThreads;
@@ -51,12 +51,12 @@ struct Shared {
   uint32_t bitmap[kWords];          // selected positions
   uint32_t tie_key[kTieCap];
   int tie_pos[kTieCap];
-  unsigned cnt[kRadix];             // radix pass histograms
+  unsigned cnt[4][kRadix];          // one histogram per radix pass (all cleared up front)
   unsigned warp_tot[kWarps];
   unsigned n_tie, n_above;
   int bin_b;                        // threshold bin
   unsigned above_b;                 // keys in bins above it (from the histogram)
-  unsigned sel_digit, sel_rem;      // result of a radix pass
+  unsigned sel_digit, sel_rem, sel_cnt;  // result of a radix pass
   unsigned scan_total;              // block_exclusive's total
 };
 
@@ -72,14 +72,14 @@ __device__ __forceinline__ unsigned block_exclusive(unsigned v, unsigned *total,
   if (lane == 31) sm.warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    unsigned w = sm.warp_tot[lane];
+    const unsigned w = lane < kWarps ? sm.warp_tot[lane] : 0u;
     unsigned s = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned y = __shfl_up_sync(0xFFFFFFFFu, s, o);
       if (lane >= o) s += y;
     }
-    sm.warp_tot[lane] = s - w;                    // exclusive over warps
+    if (lane < kWarps) sm.warp_tot[lane] = s - w;  // exclusive over warps
     if (lane == 31) sm.scan_total = s;
   }
   __syncthreads();
@@ -89,20 +89,39 @@ __device__ __forceinline__ unsigned block_exclusive(unsigned v, unsigned *total,
   return ex;
 }
 
-// Among the counts sm.cnt[0..kRadix) find, scanning from `from_top` ? the highest
-// digit : the lowest, the digit d at which the running count reaches `need`.
-// Writes d and the count strictly before d (in scan order) to sm.sel_digit/sel_rem.
-__device__ __forceinline__ void find_digit(unsigned need, bool from_top, Shared &sm) {
-  const int tid = threadIdx.x;                    // one digit per thread (kRadix == kThreads)
-  const int d = from_top ? kRadix - 1 - tid : tid;
-  unsigned tot;
-  const unsigned c = sm.cnt[d];
-  const unsigned before = block_exclusive(c, &tot, sm);
-  if (before < need && before + c >= need) {
-    sm.sel_digit = (unsigned)d;
-    sm.sel_rem = before;
+// One warp: among the counts c[0..kRadix), scanning from `from_top` ? the highest
+// digit : the lowest, the digit d at which the running count reaches `need`. Writes
+// d, the count strictly before d (in scan order) and c[d] to sm.sel_*.
+__device__ __forceinline__ void find_digit_warp(const unsigned *c, unsigned need, bool from_top, Shared &sm) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kRadix / 32;
+  unsigned mine = 0;
+#pragma unroll 8
+  for (int j = 0; j < kPer; ++j) {  // lane l takes digits l*32 .. l*32+31 in scan order
+    const int i = lane * kPer + j;
+    mine += c[from_top ? kRadix - 1 - i : i];
   }
-  __syncthreads();
+  unsigned incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  unsigned before = incl - mine;
+  if (before < need && incl >= need) {  // the crossing lane walks its own digits again
+    for (int j = 0; j < kPer; ++j) {
+      const int i = lane * kPer + j;
+      const int d = from_top ? kRadix - 1 - i : i;
+      const unsigned v = c[d];
+      if (before + v >= need) {
+        sm.sel_digit = (unsigned)d;
+        sm.sel_rem = before;
+        sm.sel_cnt = v;
+        break;
+      }
+      before += v;
+    }
+  }
 }
 
 struct CandParams {
@@ -121,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Shared &sm = *reinterpret_cast<Shared *>(smem_raw);
   pdl_prologue();
-  const int t = blockIdx.x, tid = threadIdx.x;
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int *out = p.idx + (long long)t * p.k;
   const RowPos rp = row_position(p.L, t);
   const long long n = (long long)rp.pos + 1;      // keys of the row
@@ -131,7 +150,15 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
     return;
   }
   const unsigned m = (unsigned)min((long long)p.k, n);
-  for (int w = tid; w < kWords; w += kThreads) sm.bitmap[w] = 0u;
+  const int nw = (int)((n + 31) >> 5);             // bitmap words in use
+  // the row's histogram, this thread's 8 bins from the top down
+  const unsigned *h = p.hist + (long long)t * kBins;
+  const int b_hi = kBins - 1 - tid * kBinsPerThread;
+  const uint4 ha = __ldg(reinterpret_cast<const uint4 *>(h + b_hi - 7));
+  const uint4 hb = __ldg(reinterpret_cast<const uint4 *>(h + b_hi - 3));
+  const unsigned hv[kBinsPerThread] = {hb.w, hb.z, hb.y, hb.x, ha.w, ha.z, ha.y, ha.x};
+  for (int w = tid; w < nw; w += kThreads) sm.bitmap[w] = 0u;
+  for (int i = tid; i < 4 * kRadix; i += kThreads) (&sm.cnt[0][0])[i] = 0u;
   if (tid == 0) {
     sm.n_tie = 0;
     sm.n_above = 0;
@@ -139,14 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   }
 
   // ---- 1. threshold bin: the highest b with at least m keys in bins >= b
-  const unsigned *h = p.hist + (long long)t * kBins;
-  unsigned hv[kBinsPerThread], mine = 0;
-  const int b_hi = kBins - 1 - tid * kBinsPerThread;  // this thread's bins, from the top down
+  unsigned mine = 0;
 #pragma unroll
-  for (int j = 0; j < kBinsPerThread; ++j) {
-    hv[j] = __ldg(h + b_hi - j);
-    mine += hv[j];
-  }
+  for (int j = 0; j < kBinsPerThread; ++j) mine += hv[j];
   unsigned total;
   unsigned above = block_exclusive(mine, &total, sm);  // keys in bins above this thread's
   if (total < m) {  // the histogram does not count the row's keys
@@ -174,7 +196,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   }
   const float *cs = p.score + (long long)t * p.cap;
   const int *cp = p.pos + (long long)t * p.cap;
-  const int lane = tid & 31;
   const unsigned lt = (1u << lane) - 1u;
   // every lane of a warp runs the same iterations, so the counters take one
   // shared-memory atomic per warp (ballot and population count), not one per key;
@@ -233,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
     return;
   }
 
-  // ---- 3. exact ranking inside bin B: key bits 19..10, 9..0, then position
+  // ---- 3. exact ranking inside bin B: key bits 19..10, 9..0, then (only when
+  // more keys equal the threshold key than are taken) the position, lowest first
   const bool staged = n_tie <= kTieCap;
   auto for_ties = [&](auto f) {  // every (key, position) of bin B, this thread's share
     if (staged) {
@@ -249,41 +271,43 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   int pstar = kMaxPos - 1;  // largest selected position among keys equal to kstar
   if (need_ties < n_tie) {
     uint32_t prefix = (uint32_t)B << 20;
-    unsigned need = need_ties;
+    unsigned need = need_ties, at_kstar = 0;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
       const int shift = pass == 0 ? 10 : 0;
       const uint32_t pmask = pass == 0 ? 0xFFF00000u : 0xFFFFFC00u;
-      sm.cnt[tid] = 0;
-      __syncthreads();
+      unsigned *c = sm.cnt[pass];
       for_ties([&](uint32_t key, int) {
-        if ((key & pmask) == prefix) atomicAdd(&sm.cnt[(key >> shift) & (kRadix - 1)], 1u);
+        if ((key & pmask) == prefix) atomicAdd(&c[(key >> shift) & (kRadix - 1)], 1u);
       });
       __syncthreads();
-      find_digit(need, true, sm);
+      if (warp == 0) find_digit_warp(c, need, true, sm);
+      __syncthreads();
       prefix |= sm.sel_digit << shift;
       need -= sm.sel_rem;
-      __syncthreads();
+      at_kstar = sm.sel_cnt;
     }
     kstar = prefix;  // need = how many keys equal to kstar are taken (lowest positions first)
+    if (need < at_kstar) {
 #pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {  // positions < 2^18 in two 9-bit digits
-      const int shift = pass == 0 ? 9 : 0;
-      sm.cnt[tid] = 0;
-      __syncthreads();
-      for_ties([&](uint32_t key, int s) {
-        const bool in = key == kstar && (pass == 0 || (s >> 9) == (pstar >> 9));
-        if (in) atomicAdd(&sm.cnt[(s >> shift) & 511], 1u);
-      });
-      __syncthreads();
-      find_digit(need, false, sm);
-      if (pass == 0) {
-        pstar = (int)(sm.sel_digit << 9) | 511;
-      } else {
-        pstar = (pstar & ~511) | (int)sm.sel_digit;
+      for (int pass = 0; pass < 2; ++pass) {  // positions < 2^18 in two 9-bit digits
+        const int shift = pass == 0 ? 9 : 0;
+        unsigned *c = sm.cnt[2 + pass];
+        const int phi = pstar >> 9;
+        for_ties([&](uint32_t key, int s) {
+          const bool in = key == kstar && (pass == 0 || (s >> 9) == phi);
+          if (in) atomicAdd(&c[(s >> shift) & 511], 1u);
+        });
+        __syncthreads();
+        if (warp == 0) find_digit_warp(c, need, false, sm);
+        __syncthreads();
+        if (pass == 0) {
+          pstar = (int)(sm.sel_digit << 9) | 511;
+        } else {
+          pstar = (pstar & ~511) | (int)sm.sel_digit;
+        }
+        need -= sm.sel_rem;
       }
-      need -= sm.sel_rem;
-      __syncthreads();
     }
   } else {
     kstar = 0;  // every tie is taken
@@ -295,7 +319,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   __syncthreads();
 
   // ---- 4. ascending emission, then padding
-  const int nw = (int)((n + 31) >> 5);
   const int w0 = tid * kWordsPerThread;
   unsigned pc = 0;
 #pragma unroll
