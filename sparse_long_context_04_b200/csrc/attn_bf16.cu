@@ -347,124 +347,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the splits of each row: with o_c the split's output already divided by its
-// own sum l_c, out = sum_c w_c o_c with w_c = e^{m_c - M} l_c / sum_c' e^{m_c' - M} l_c'
-// (per head), and lse = M + ln sum_c e^{m_c - M} l_c.
-// One CTA per (row, 32 output values), 128 threads. Thread (value v, heads 32g ..
-// 32g+31) reads 16 bytes (8 heads) per load from the head-minor partials, so that a
-// warp reads 2 KB of consecutive memory per instruction. The first batch of splits
-// is requested before anything else, while each thread (one head) turns the
-// splits' (max, sum) pairs into weights in shared memory; a split without keys has
-// weight 0 and its partial (never written) is loaded but not used. The sums are
-// transposed through shared memory so that each head's 32 values leave as 16-byte
-// stores.
-constexpr int kMergeVals = 32;
-constexpr int kMergeThreads = 128;   // 32 values x 4 head groups
-constexpr int kMergeBatch = 8;       // splits whose loads are in flight together
-constexpr int kMergeMaxSplits = 64;  // k <= 16384 at 256 keys per split
-
-size_t merge_smem_bytes(int splits) {
-  return (size_t)kH * (kMergeVals + 1) * 4 + (size_t)splits * kH * 4 + (size_t)splits * 4;
-}
-
-__device__ __forceinline__ void merge_load(const __half *src, int c0, int splits, uint4 (&raw)[kMergeBatch][4]) {
-#pragma unroll
-  for (int u = 0; u < kMergeBatch; ++u) {
-    const int c = c0 + u;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      raw[u][q] = c < splits ? __ldcs(reinterpret_cast<const uint4 *>(src + (long long)c * (kDv * kH)) + q)
-                             : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-__global__ void __launch_bounds__(kMergeThreads)
-    attn_merge_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
-                      __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-  extern __shared__ __align__(16) float merge_smem[];
-  float(*s_sum)[kMergeVals + 1] = reinterpret_cast<float(*)[kMergeVals + 1]>(merge_smem);  // [kH]: transposed sums
-  float(*s_w)[kH] = reinterpret_cast<float(*)[kH]>(merge_smem + kH * (kMergeVals + 1));    // [splits]: weights
-  int *s_live = reinterpret_cast<int *>(merge_smem + kH * (kMergeVals + 1) + splits * kH);  // the split has keys
+// Merge the splits of each (row, head) for 8 output values per CTA, one thread per
+// head. With O_c the split's output already divided by its sum l_c:
+// out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c.
+constexpr int kCombVals = 8;
+__global__ void __launch_bounds__(128)
+    attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
+                        __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   pdl_prologue();
-  const int t = blockIdx.x, v0 = blockIdx.y * kMergeVals, tid = threadIdx.x;
-  const int vi = tid >> 2, g = tid & 3;  // value v0 + vi, heads 32g .. 32g+31
-  const __half *src = o_part + (long long)t * splits * (kDv * kH) + (long long)(v0 + vi) * kH + 32 * g;
-  uint4 raw[kMergeBatch][4];
-  merge_load(src, 0, splits, raw);  // in flight while the weights are formed
-  {
-    const int h = tid;  // one head per thread for the weights
-    const float2 *ml = ml_part + (long long)t * splits * kH + h;
-    float2 first[kMergeBatch];
-    float M = -INFINITY;
-    for (int c0 = 0; c0 < splits; c0 += kMergeBatch) {
-      float2 mv[kMergeBatch];
-#pragma unroll
-      for (int u = 0; u < kMergeBatch; ++u)
-        mv[u] = c0 + u < splits ? ml[(c0 + u) * kH] : make_float2(-INFINITY, 0.f);
-#pragma unroll
-      for (int u = 0; u < kMergeBatch; ++u) {
-        if (c0 == 0) first[u] = mv[u];
-        if (mv[u].y > 0.f) M = fmaxf(M, mv[u].x);
-      }
-    }
-    float L = 0.f;
-    for (int c0 = 0; c0 < splits; c0 += kMergeBatch) {
-      float2 mv[kMergeBatch];
-#pragma unroll
-      for (int u = 0; u < kMergeBatch; ++u)
-        mv[u] = c0 == 0 ? first[u] : (c0 + u < splits ? ml[(c0 + u) * kH] : make_float2(-INFINITY, 0.f));
-#pragma unroll
-      for (int u = 0; u < kMergeBatch; ++u) {
-        if (c0 + u >= splits) break;
-        const float w = mv[u].y > 0.f ? __expf(mv[u].x - M) * mv[u].y : 0.f;
-        s_w[c0 + u][h] = w;
-        L += w;
-        if (h == 0) s_live[c0 + u] = mv[u].y > 0.f;
-      }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int c = 0; c < splits; ++c) s_w[c][h] *= inv;
-    if (lse && blockIdx.y == 0) lse[(long long)t * kH + h] = L > 0.f ? M + logf(L) : -INFINITY;
+  const int t = blockIdx.x, d0 = blockIdx.y * kCombVals, h = threadIdx.x;
+  const float2 *ml = ml_part + (long long)t * splits * kH + h;
+  float M = -INFINITY;
+  for (int c = 0; c < splits; ++c) {
+    const float2 v = ml[c * kH];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
   }
-  __syncthreads();
-  float acc[32];
+  float acc[kCombVals];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-  for (int c0 = 0; c0 < splits; c0 += kMergeBatch) {
-    if (c0 > 0) merge_load(src, c0, splits, raw);
+  for (int x = 0; x < kCombVals; ++x) acc[x] = 0.f;
+  float Lsum = 0.f;
+  const __half *ob = o_part + (long long)t * splits * (kDv * kH) + (long long)d0 * kH + h;
+  for (int c0 = 0; c0 < splits; c0 += 4) {
+    float vals[4][kCombVals], wgt[4];
 #pragma unroll
-    for (int u = 0; u < kMergeBatch; ++u) {
+    for (int u = 0; u < 4; ++u) {  // all loads of four splits in flight together
       const int c = c0 + u;
-      if (c >= splits) break;
-      if (!s_live[c]) continue;  // no keys: its partial was never written
-      const float4 *w4 = reinterpret_cast<const float4 *>(&s_w[c][32 * g]);
+      const float2 v = c < splits ? ml[c * kH] : make_float2(-INFINITY, 0.f);
+      wgt[u] = v.y > 0.f ? __expf(v.x - M) * v.y : 0.f;  // the split's share before normalising
+      Lsum += wgt[u];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __half2 *hv = reinterpret_cast<const __half2 *>(&raw[u][q]);
-        const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
-        const float2 f0 = __half22float2(hv[0]), f1 = __half22float2(hv[1]);
-        const float2 f2 = __half22float2(hv[2]), f3 = __half22float2(hv[3]);
-        acc[8 * q + 0] = fmaf(wa.x, f0.x, acc[8 * q + 0]);
-        acc[8 * q + 1] = fmaf(wa.y, f0.y, acc[8 * q + 1]);
-        acc[8 * q + 2] = fmaf(wa.z, f1.x, acc[8 * q + 2]);
-        acc[8 * q + 3] = fmaf(wa.w, f1.y, acc[8 * q + 3]);
-        acc[8 * q + 4] = fmaf(wb.x, f2.x, acc[8 * q + 4]);
-        acc[8 * q + 5] = fmaf(wb.y, f2.y, acc[8 * q + 5]);
-        acc[8 * q + 6] = fmaf(wb.z, f3.x, acc[8 * q + 6]);
-        acc[8 * q + 7] = fmaf(wb.w, f3.y, acc[8 * q + 7]);
-      }
+      for (int x = 0; x < kCombVals; ++x)
+        vals[u][x] = wgt[u] != 0.f ? __half2float(__ldcs(ob + (long long)c * (kDv * kH) + x * kH)) : 0.f;
     }
-  }
 #pragma unroll
-  for (int i = 0; i < 32; ++i) s_sum[32 * g + i][vi] = acc[i];
-  __syncthreads();
-  // each head's 32 values as four 16-byte stores: thread (head, quarter)
-  for (int e = tid; e < kH * 4; e += kMergeThreads) {
-    const int h = e >> 2, qv = e & 3;
-    const float *r = &s_sum[h][8 * qv];
-    *reinterpret_cast<uint4 *>(out + ((long long)t * kH + h) * kDv + v0 + 8 * qv) =
-        make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7]));
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int x = 0; x < kCombVals; ++x) acc[x] = fmaf(wgt[u], vals[u][x], acc[x]);
   }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  *reinterpret_cast<uint4 *>(out + ((long long)t * kH + h) * kDv + d0) =
+      make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                 pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+  if (lse && blockIdx.y == 0) lse[(long long)t * kH + h] = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
 }
 
 // ------------------------------------------------------------------ host
@@ -561,11 +485,7 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     p.L.row0 = L.row0 + r0;
     err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)merge_smem_bytes(kMergeMaxSplits));
-    if (err != cudaSuccess) return err;
-    err = launch_kernel(attn_merge_kernel, dim3(nr, kDv / kMergeVals), dim3(kMergeThreads),
-                        merge_smem_bytes(pl.splits), stream, 0,
+    err = launch_kernel(attn_combine_kernel, dim3(nr, kDv / kCombVals), dim3(128), 0, stream, 0,
                         static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                         static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
                         lse ? lse + (size_t)r0 * kH : nullptr);
@@ -648,11 +568,7 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   p.e = e;
   err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)merge_smem_bytes(kMergeMaxSplits));
-  if (err != cudaSuccess) return err;
-  return launch_kernel(attn_merge_kernel, dim3(T, kDv / kMergeVals), dim3(kMergeThreads), merge_smem_bytes(pl.splits),
-                       stream, 0,
+  return launch_kernel(attn_combine_kernel, dim3(T, kDv / kCombVals), dim3(128), 0, stream, 0,
                        static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                        static_cast<__nv_bfloat16 *>(out), lse);
 }
