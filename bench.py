@@ -174,6 +174,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill FP8 indexer measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other four workloads (stages, dsa_forward, roofline fractions)")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip timing the sparse-attention backward on the step's selection")
     ap.add_argument("--all-configs", action="store_true",
@@ -205,7 +207,8 @@ def main():
 
     if args.all_configs:
         if rank == 0:
-            all_configs(dev, G, D, W, only=args.only)
+            for line in all_configs(dev, G, D, W, only=args.only).values():
+                print(json.dumps(dict(mode="all_configs", **line)), flush=True)
         X.finish()
         return
 
@@ -471,6 +474,13 @@ def main():
     # the dense FP8 peak measured here
     fp8_tf = measure_fp8_peak(dev) if not args.no_prefill else None
     pf = prefill_indexer(args, dev, G, D, W, fp8_measured=fp8_tf) if not args.no_prefill else None
+    # ---- every other workload through the library: stages, dsa_forward, roofline fractions
+    cfgs = None
+    if not args.no_configs and rank == 0:
+        del dc, scores, hist, cand_s, cand_p, cand_n, ws
+        torch.cuda.empty_cache()
+        cfgs = all_configs(dev, G, D, W, fp8_measured=fp8_tf,
+                           names=[n for n in CONFIG_REPS if n != WORKLOAD])
     sampler.stop_flag.set()
     sampler.join()
     if D.dsa_get_device_error() != D.DSA_OK:
@@ -529,6 +539,7 @@ def main():
                                "algorithmic_bytes": ab["topk"] + ab["attn"]},
         "step_roofline": {"achieved": step_gbs, "frac": step_gbs / hbm, "algorithmic_bytes": sum(ab.values())},
         "fp8_indexer_prefill": pf,
+        "configs": cfgs,
         "fp8_peak_tflops": {"measured": fp8_tf, "datasheet": FP8_DATASHEET_TFLOPS,
                             "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10, CUDA events"},
         "e2e": {"value": X.job_rate(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
@@ -659,82 +670,95 @@ def prefill_indexer(args, dev, G, D, W, reps=20, fp8_measured=None):
             "datasheet_tflops": FP8_DATASHEET_TFLOPS, "kernel": "indexer_fp8_kernel (prefill, N=256)"}
 
 
-def all_configs(dev, G, D, W, only=None):
-    """Every workload once: per-stage CUDA-event times (each stage called on its own),
-    the composed dsa_forward, tokens/s and each stage against its roofline (the larger
-    of bytes / measured HBM and flops / the dtype's peak). One JSON line per workload."""
+def config_line(spec, reps, dev, G, D, W, hbm, bf16, fp8):
+    """One workload through the library: per-stage CUDA-event times (each stage
+    called on its own over every row, L2 warm), the composed dsa_forward, tokens/s
+    and each stage against its roofline (the larger of algorithmic bytes / measured
+    HBM bandwidth and flops / the dtype's measured dense peak)."""
+    inp = W.make_inputs(spec, big_q_device=dev)
+    dc = G.to_device(inp, dev)
+    T, s = dc.T, spec
+    pos = inp.pos.to(torch.int64)
+    n_pairs = int((pos + 1).sum())
+    n_sel = int(torch.clamp(pos + 1, max=s.k).sum())
+    lens = [int(x) for x in inp.seq_lens.tolist()]
+    scores = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, s.k), dtype=torch.int32, device=dev)
+    out = torch.empty((T, s.H, s.Dv), dtype=dc.q.dtype, device=dev)
+    lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
+    wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
+    ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
+    stages = {
+        "indexer": lambda: D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout, scores),
+        "topk": lambda: D.dsa_topk(scores, s.k, dc.layout, idx),
+        "attention": lambda: D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws),
+    }
+    ms = {}
+    for name, fn in stages.items():
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms[name] = e0.elapsed_time(e1) / reps
+    del scores
+    fw = G.Forward(dc, keep_idx=False)
+    for _ in range(2):
+        fw()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fw()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    fwd_ms = e0.elapsed_time(e1) / reps
+    if D.dsa_get_device_error() != D.DSA_OK:
+        raise RuntimeError(f"device error on {spec.name}")
+    line = {"workload": spec.name, "query_rows": T, "tokens_per_s": T / (fwd_ms / 1e3), "forward_ms": fwd_ms,
+            "stages_ms": ms, "dtype": "fp32" if not s.fp8 else "e4m3 indexer + bf16 attention"}
+    if s.fp8:
+        kbytes = sum(lens) * (s.d_I + 4) + T * (s.H_I * s.d_I + 4 + 4 * s.H_I)
+        roof = {
+            "indexer": max((kbytes + n_pairs * 4) / hbm / 1e6, 2 * s.H_I * s.d_I * n_pairs / fp8 / 1e9),
+            "topk": (n_pairs * 4 + T * s.k * 4) / hbm / 1e6,
+            "attention": max((n_sel * s.Dk * 2 + T * s.H * (s.Dk + s.Dv) * 2 + T * s.H * 4) / hbm / 1e6,
+                             2 * s.H * (s.Dk + s.Dv) * n_sel / bf16 / 1e9),
+        }
+        line["roofline_ms"] = roof
+        line["frac"] = {k: roof[k] / ms[k] for k in roof}
+        line["forward_frac"] = sum(roof.values()) / fwd_ms
+        line["bound"] = "hbm" if s.mode == "decode" else "tensor (fp8 indexer, bf16 attention)"
+    del dc, idx, out, lse, ws, fw, inp
+    torch.cuda.empty_cache()
+    return line
+
+
+CONFIG_REPS = {"tiny_fp32_prefill_L256": 20, "decode_b32_ctx32k": 50, "prefill_L8192": 5,
+               "prefill_2x32768_ar1": 2, "paged_decode_b16_ctx96k_128k": 50}
+
+
+def all_configs(dev, G, D, W, only=None, fp8_measured=None, names=None):
+    """Every workload once (or `only`): a dict name -> config_line."""
     hbm, _ = peaks()
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             bf16 = float(json.load(f)["bf16_tflops"])
     except Exception:
         bf16 = 1590.0
-    fp8, fp8_src = fp8_peak(measure_fp8_peak(dev))
-    for spec, reps in ((W.TINY, 20), (W.DECODE_32K, 50), (W.PREFILL_8K, 5), (W.PREFILL_2X32K, 2),
-                       (W.PAGED_DECODE_128K, 50)):
-        if only and spec.name != only:
+    fp8, fp8_src = fp8_peak(fp8_measured if fp8_measured else measure_fp8_peak(dev))
+    res = {}
+    for spec in (W.TINY, W.DECODE_32K, W.PREFILL_8K, W.PREFILL_2X32K, W.PAGED_DECODE_128K):
+        if (only and spec.name != only) or (names is not None and spec.name not in names):
             continue
-        inp = W.make_inputs(spec)
-        dc = G.to_device(inp, dev)
-        T, s = dc.T, spec
-        pos = inp.pos.to(torch.int64)
-        n_pairs = int((pos + 1).sum())
-        n_sel = int(torch.clamp(pos + 1, max=s.k).sum())
-        lens = [int(x) for x in inp.seq_lens.tolist()]
-        scores = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
-        idx = torch.empty((T, s.k), dtype=torch.int32, device=dev)
-        out = torch.empty((T, s.H, s.Dv), dtype=dc.q.dtype, device=dev)
-        lse = torch.empty((T, s.H), dtype=torch.float32, device=dev)
-        wsn = D.dsa_sparse_mqa_attn_workspace_size(T, s.H, s.Dv, s.k, dc.q)
-        ws = torch.empty(max(wsn, 256), dtype=torch.uint8, device=dev)
-        stages = {
-            "indexer": lambda: D.dsa_indexer_scores(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.layout,
-                                                    scores),
-            "topk": lambda: D.dsa_topk(scores, s.k, dc.layout, idx),
-            "attention": lambda: D.dsa_sparse_mqa_attn(dc.q, dc.kv, idx, dc.layout, out, lse, s.softmax_scale, ws),
-        }
-        ms = {}
-        for name, fn in stages.items():
-            for _ in range(2):
-                fn()
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(reps):
-                fn()
-            e1.record()
-            torch.cuda.synchronize(dev)
-            ms[name] = e0.elapsed_time(e1) / reps
-        fw = G.Forward(dc, keep_idx=False)
-        for _ in range(2):
-            fw()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            fw()
-        e1.record()
-        torch.cuda.synchronize(dev)
-        fwd_ms = e0.elapsed_time(e1) / reps
-        if D.dsa_get_device_error() != D.DSA_OK:
-            raise RuntimeError(f"device error on {spec.name}")
-        line = {"mode": "all_configs", "workload": spec.name, "query_rows": T, "tokens_per_s": T / (fwd_ms / 1e3),
-                "forward_ms": fwd_ms, "stages_ms": ms, "dtype": "fp32" if not s.fp8 else "e4m3 indexer + bf16 attention"}
-        if s.fp8:
-            kbytes = sum(lens) * (s.d_I + 4) + T * (s.H_I * s.d_I + 4 + 4 * s.H_I)
-            roof = {
-                "indexer": max((kbytes + n_pairs * 4) / hbm / 1e6, 2 * s.H_I * s.d_I * n_pairs / fp8 / 1e9),
-                "topk": (n_pairs * 4 + T * s.k * 4) / hbm / 1e6,
-                "attention": max((n_sel * s.Dk * 2 + T * s.H * (s.Dk + s.Dv) * 2 + T * s.H * 4) / hbm / 1e6,
-                                 2 * s.H * (s.Dk + s.Dv) * n_sel / bf16 / 1e9),
-            }
-            line["roofline_ms"] = roof
-            line["frac"] = {k: roof[k] / ms[k] for k in roof}
-            line["forward_frac"] = sum(roof.values()) / fwd_ms
-            line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": bf16, "fp8_tflops": fp8, "fp8_source": fp8_src}
-        print(json.dumps(line), flush=True)
-        del dc, scores, idx, out, lse, ws, fw
-        torch.cuda.empty_cache()
+        line = config_line(spec, CONFIG_REPS[spec.name], dev, G, D, W, hbm, bf16, fp8)
+        line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": bf16, "fp8_tflops": fp8, "fp8_source": fp8_src}
+        res[spec.name] = line
+    return res
 
 
 def run_reference(args, world, rank):

@@ -186,8 +186,13 @@ def draw_lens(spec: Spec) -> list:
     return [int(v) for v in g.integers(lo, hi + 1, size=spec.batch)]
 
 
-def make_inputs(spec: Spec) -> Inputs:
-    """Build every input tensor of `spec` on the host (torch CPU tensors)."""
+def make_inputs(spec: Spec, big_q_device=None) -> Inputs:
+    """Build every input tensor of `spec` on the host (torch CPU tensors).
+
+    big_q_device: for the large prefill workloads, whose iid query block is
+    gigabytes, draw that block directly on this device (torch's generator, seeded
+    from the workload seed; N(0,1) rounded to bf16) instead of on the host. Used by
+    the benchmark only; its values differ from the host stream's."""
     lens = draw_lens(spec)
     B = spec.batch
     if spec.mode == "decode":
@@ -248,7 +253,11 @@ def make_inputs(spec: Spec) -> Inputs:
     # ---- encode ----
     if spec.fp8:
         q_idx, q_scale = encode_e4m3_per_token(qI)
-        if big_q:
+        if big_q and big_q_device is not None:
+            g = torch.Generator(device=big_q_device).manual_seed(zlib.crc32(b"q") ^ (seed & 0xFFFFFFFF))
+            q_t = torch.randn((T, spec.H, spec.Dk), generator=g, device=big_q_device,
+                              dtype=torch.float32).to(torch.bfloat16)
+        elif big_q:
             q_t = torch.empty((T, spec.H, spec.Dk), dtype=torch.bfloat16)
             for r0 in range(0, T, _CHUNK_ROWS):
                 r1 = min(T, r0 + _CHUNK_ROWS)

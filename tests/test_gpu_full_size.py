@@ -4,7 +4,10 @@ benchmark times), on sampled query rows the oracle computes one by one:
   - top-k: bit-exact against the oracle's selection on the GPU's own scores,
     and equal to the selection dsa_forward made,
   - attention: output and log-sum-exp within 2e-2, recomputed on the GPU's indices.
-Sampled rows include the short-row boundary (pos = k-1, k) and sequence edges."""
+Sampled rows include the short-row boundary (pos = k-1, k) and sequence edges.
+On the prefill workloads the selection is also checked on every row: the GPU's
+scores of each chunk of 4096 rows (a prefill call of its own over the same cache)
+against the oracle's top-k of those scores, bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -68,7 +71,37 @@ def _run(name):
         e1 = np.abs(o_np[r] - o).max()
         e2 = np.abs(l_np[r] - l).max()
         assert e1 <= TOL and e2 <= TOL, (name, t, e1, e2)
+    if spec.mode == "prefill":
+        assert _topk_every_row(dc, idx) == inp.T
     return len(rows)
+
+
+def _topk_every_row(dc, idx, chunk=4096):
+    """Every prefill row's selection against the oracle's top-k of the GPU's scores.
+    Rows r0..r1-1 of sequence b (positions p0..p1-1) are scored as a prefill call of
+    their own: one sequence of length p1 whose last r1-r0 tokens are the queries."""
+    inp, spec = dc.inp, dc.inp.spec
+    dev = dc.q.device
+    cu = inp.cu_q.tolist()
+    pos = inp.pos.numpy()
+    checked = 0
+    for b in range(len(cu) - 1):
+        for r0 in range(cu[b], cu[b + 1], chunk):
+            r1 = min(cu[b + 1], r0 + chunk)
+            lay = D.Layout(torch.tensor([int(pos[r1 - 1]) + 1], dtype=torch.int32, device=dev), dc.layout.c.n_max,
+                           torch.tensor([0, r1 - r0], dtype=torch.int32, device=dev))
+            scores = torch.empty((r1 - r0, dc.ld), dtype=torch.float32, device=dev)
+            D.dsa_indexer_scores(dc.q_idx[r0:r1], dc.q_scale[r0:r1], dc.k_idx[b:b + 1], dc.k_scale[b:b + 1],
+                                 dc.w[r0:r1], lay, scores)
+            torch.cuda.synchronize()
+            assert D.dsa_get_device_error() == D.DSA_OK
+            want = O.topk_rows(scores.cpu().numpy(), (pos[r0:r1] + 1).astype(np.int32), spec.k)
+            got = idx[r0:r1].cpu().numpy()
+            bad = np.nonzero((got != want).any(axis=1))[0]
+            assert bad.size == 0, (spec.name, int(r0 + bad[0]))
+            checked += r1 - r0
+            del scores
+    return checked
 
 
 def test_full_decode_b32_ctx32k():
