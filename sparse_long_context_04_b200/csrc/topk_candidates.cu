@@ -34,7 +34,6 @@ constexpr int kBins = 4096;                   // top 12 bits of the order key
 constexpr int kBinsPerThread = kBins / kThreads;
 constexpr int kMaxPos = 262144;               // positions per row (bitmap bits)
 constexpr int kWords = kMaxPos / 32;
-constexpr int kWordsPerThread = kWords / kThreads;
 constexpr int kTieCap = 12288;                // tie entries staged in shared memory
 constexpr int kRadix = 1024;                  // bins of the later radix passes
 
@@ -197,11 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   const float *cs = p.score + (long long)t * p.cap;
   const int *cp = p.pos + (long long)t * p.cap;
   const unsigned lt = (1u << lane) - 1u;
-  // every lane of a warp runs the same iterations, so the counters take one
-  // shared-memory atomic per warp (ballot and population count), not one per key;
-  // each lane loads kU candidates before it looks at any, so that the loads'
-  // latencies overlap
+  // Every lane of a warp runs the same iterations. Each lane loads kU candidates
+  // before it looks at any, so that the loads' latencies overlap; a warp reserves
+  // its ties' slots with one shared-memory atomic per kU x 32 candidates, and the
+  // keys above B are counted per thread and summed once at the end.
   constexpr int kU = 8;
+  unsigned my_above = 0;
   for (long long i0 = (long long)(tid - lane) * kU; i0 < cnt; i0 += (long long)kThreads * kU) {
     float sc[kU];
     int ps[kU];
@@ -211,12 +211,13 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
       sc[j] = i < cnt ? __ldg(cs + i) : 0.f;
       ps[j] = i < cnt ? __ldg(cp + i) : 0;
     }
+    unsigned tie_bits = 0, tmask[kU], n_tie_w = 0;
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const long long i = i0 + j * 32 + lane;
-      bool is_above = false, is_tie = false;
       const uint32_t key = order_key(sc[j]);
       const int s = ps[j];
+      bool is_above = false, is_tie = false;
       if (i < cnt) {
         const int bin = (int)(key >> 20);
         if (bin >= B) {
@@ -229,22 +230,31 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
         }
       }
       if (is_above) atomicOr(&sm.bitmap[s >> 5], 1u << (s & 31));
-      const unsigned ma = __ballot_sync(0xFFFFFFFFu, is_above), mt = __ballot_sync(0xFFFFFFFFu, is_tie);
+      my_above += is_above;
+      tmask[j] = __ballot_sync(0xFFFFFFFFu, is_tie);
+      tie_bits |= (unsigned)is_tie << j;
+      n_tie_w += __popc(tmask[j]);
+    }
+    if (n_tie_w) {
       unsigned tb = 0;
-      if (lane == 0) {
-        if (ma) atomicAdd(&sm.n_above, (unsigned)__popc(ma));
-        if (mt) tb = atomicAdd(&sm.n_tie, (unsigned)__popc(mt));
-      }
+      if (lane == 0) tb = atomicAdd(&sm.n_tie, n_tie_w);
       tb = __shfl_sync(0xFFFFFFFFu, tb, 0);
-      if (is_tie) {
-        const unsigned slot = tb + __popc(mt & lt);
-        if (slot < kTieCap) {
-          sm.tie_key[slot] = key;
-          sm.tie_pos[slot] = s;
+#pragma unroll
+      for (int j = 0; j < kU; ++j) {
+        if ((tie_bits >> j) & 1u) {
+          const unsigned slot = tb + __popc(tmask[j] & lt);
+          if (slot < kTieCap) {
+            sm.tie_key[slot] = order_key(sc[j]);
+            sm.tie_pos[slot] = ps[j];
+          }
         }
+        tb += __popc(tmask[j]);
       }
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_above += __shfl_xor_sync(0xFFFFFFFFu, my_above, o);
+  if (lane == 0 && my_above) atomicAdd(&sm.n_above, my_above);
   __syncthreads();
   const unsigned n_tie = sm.n_tie;
   // every key in bins >= B must have been a candidate: the counts must agree
@@ -318,25 +328,50 @@ __global__ void __launch_bounds__(kThreads, 1) topk_candidates_kernel(const Cand
   });
   __syncthreads();
 
-  // ---- 4. ascending emission, then padding
-  const int w0 = tid * kWordsPerThread;
-  unsigned pc = 0;
+  // ---- 4. ascending emission, then padding. Warp w takes a contiguous block of
+  // bitmap words, 32 at a time (one per lane): its total first, then, after a scan
+  // of the warps' totals, each lane writes its word's positions at its prefix.
+  const int per_w = (nw + kWarps - 1) / kWarps;
+  const int wb0 = min(nw, warp * per_w), wb1 = min(nw, wb0 + per_w);
+  unsigned wt = 0;
+  for (int w = wb0 + lane; w < wb1; w += 32) wt += __popc(sm.bitmap[w]);
 #pragma unroll
-  for (int j = 0; j < kWordsPerThread; ++j)
-    if (w0 + j < nw) pc += __popc(sm.bitmap[w0 + j]);
-  unsigned emitted;
-  unsigned off = block_exclusive(pc, &emitted, sm);
+  for (int o = 16; o > 0; o >>= 1) wt += __shfl_xor_sync(0xFFFFFFFFu, wt, o);
+  if (lane == 0) sm.warp_tot[warp] = wt;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned v = lane < kWarps ? sm.warp_tot[lane] : 0u;
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < kWarps) sm.warp_tot[lane] = incl - v;
+    if (lane == 31) sm.scan_total = incl;
+  }
+  __syncthreads();
+  const unsigned emitted = sm.scan_total;
   if (emitted != m && tid == 0) raise_error(p.e, DEV_BOUNDS, 0x905);
+  unsigned base = sm.warp_tot[warp];
+  for (int w0 = wb0; w0 < wb1; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t bits = w < wb1 ? sm.bitmap[w] : 0u;
+    const unsigned c = __popc(bits);
+    unsigned incl = c;
 #pragma unroll
-  for (int j = 0; j < kWordsPerThread; ++j) {
-    if (w0 + j >= nw) break;
-    uint32_t bits = sm.bitmap[w0 + j];
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    unsigned off = base + incl - c;
     while (bits) {
-      const int b = __ffs(bits) - 1;
+      const int bit = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (off < (unsigned)p.k) out[off] = (w0 + j) * 32 + b;
+      if (off < (unsigned)p.k) out[off] = w * 32 + bit;
       ++off;
     }
+    base += __shfl_sync(0xFFFFFFFFu, incl, 31);
   }
   for (int i = (int)emitted + tid; i < p.k; i += kThreads) out[i] = -1;
 }
