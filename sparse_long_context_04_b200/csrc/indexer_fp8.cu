@@ -547,7 +547,11 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
         cur.seek(p, s_seq, s_fseq, n_items);
         int g_seen = 0;  // query groups whose slot this warp has waited for
         bool ok = true;
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        // descriptors built once: a stage, query slot or K step moves only the start
+        // address field (16-byte units; shared addresses stay below 2^18, so adding
+        // an offset never carries out of the field)
+        const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, SW_128B);
+        const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, SW_128B);
         for (long long n = 0; n < n_items && ok; ++n) {
           const int g = cur.gcount - 1;
           const int slot = g & 1;
@@ -566,12 +570,10 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t d = tmem + (uint32_t)(ab * C::N);
+            const uint64_t ad = a_desc0 + (uint64_t)((st * C::kATile) >> 4);
+            const uint64_t bd = b_desc0 + (uint64_t)((slot * C::kBTile) >> 4);
 #pragma unroll
-            for (int ks = 0; ks < kDI / 32; ++ks) {
-              const uint64_t ad = smem_desc(a0 + st * C::kATile + ks * 32, 16, 1024, SW_128B);
-              const uint64_t bd = smem_desc(b0 + slot * C::kBTile + ks * 32, 16, 1024, SW_128B);
-              umma_f8(d, ad, bd, C::kIdesc, ks > 0);
-            }
+            for (int ks = 0; ks < kDI / 32; ++ks) umma_f8(d, ad + 2 * ks, bd + 2 * ks, C::kIdesc, ks > 0);
             umma_commit(a_empty + st);
             umma_commit(acc_full + ab);
           }
