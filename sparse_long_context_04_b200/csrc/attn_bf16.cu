@@ -8,12 +8,12 @@
 // Work unit (one CTA): query row t and a split of up to 256 of its selected
 // positions. One pass, no running rescale:
 //   1. S[128 heads, n] = Q_t[128, 576] . K_sel[n, 576]^T  — nine 64-dim chunks,
-//      Q by TMA and the selected rows gathered with cp.async into 128-byte
-//      swizzled tiles; tcgen05 kind::f16, M = 128, N = n, accumulated in TMEM.
+//      Q by a tiled TMA load and the selected rows by TMA four-row gathers into
+//      128-byte swizzled tiles; tcgen05 kind::f16, M = 128, N = n, in TMEM.
 //   2. Four warps (one head row per thread) read S from TMEM, take the row max
 //      and write P = exp(scale (S - max)) as bf16 into shared memory.
 //   3. O[128, 512] = P[128, n] . V[n, 512] with the value rows gathered again
-//      (MN-major B operand); O reuses the TMEM columns S occupied.
+//      (MN-major B operand, same tile shape); O reuses the TMEM columns S occupied.
 //   4. O (unnormalised), the row max and the row sum go to the workspace; a
 //      second kernel merges the splits of each row with log-sum-exp weights.
 #include <cuda.h>
@@ -41,16 +41,16 @@ constexpr int kVKeys = 32;                     // value rows per block
 constexpr int kVBlock = kVKeys * kDv * 2;      // 32 KiB
 constexpr int kVStages = 4;
 constexpr int kPBytes = kH * kMaxKeys * 2;     // 64 KiB
-constexpr int kProducers = 128;                // warps 0-3
+constexpr int kProducerWarps = 4;              // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per TMEM lane quadrant
 constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
-constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 8 + 256 + 1024;
+constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 4 + 256 + 1024;
 constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
 static_assert(kVStages * kVBlock <= kRing, "value blocks reuse the score ring");
 
 struct Params {
-  const __nv_bfloat16 *kv;
+  int kv_rows;        // rows of the latent cache; the gather coordinate of a padding entry
   const int *idx;
   int k;
   int splits;
@@ -80,13 +80,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                     const Params p) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   unsigned char *ring = base;
   unsigned char *sP = base + kRing;
-  long long *rows = reinterpret_cast<long long *>(sP + kPBytes);
+  int *rows = reinterpret_cast<int *>(sP + kPBytes);  // gather row of each selected entry
   uint64_t *bars = reinterpret_cast<uint64_t *>(rows + kMaxKeys);
   uint64_t *full = bars, *empty = bars + kStages;
   uint64_t *vfull = bars + 2 * kStages, *vempty = vfull + kVStages;
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         raise_error(p.e, DEV_BOUNDS, 0x501);
       }
     }
-    rows[i] = r;
+    rows[i] = r >= 0 ? (int)r : p.kv_rows;  // padding reads the zero fill past the last row
     if (r >= 0) {
       atomicMax(&s_nvalid, i + 1);
       atomicOr(&s_valid[i >> 5], 1u << (i & 31));
@@ -136,11 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full + s, kProducers + 1);
+      mbar_init(full + s, kProducerWarps);
       mbar_init(empty + s, 1);
     }
     for (int j = 0; j < kVStages; ++j) {
-      mbar_init(vfull + j, kProducers);
+      mbar_init(vfull + j, kProducerWarps);
       mbar_init(vempty + j, 1);
     }
     mbar_init(s_full, 1);
@@ -156,30 +157,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const char *kvb = reinterpret_cast<const char *>(p.kv);
 
-  if (warp < 4) {
-    // ================= producers: Q chunks by TMA, selected rows by cp.async
+  if (warp < kProducerWarps) {
+    // ================= producers: Q chunks by a tiled TMA load, selected rows by
+    // four-row TMA gathers. Warp w's lanes issue the row groups g = 4 * lane + w, after
+    // lane 0 has announced the warp's bytes on the stage barrier.
     const int tid = threadIdx.x;
-    if (tid == 0) tma_prefetch_desc(&tm_q);
+    if (tid == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kv);
+    }
+    const int groups = n / 16;  // row groups per warp and chunk (n is a multiple of 64)
     bool ok = true;
     for (int c = 0; c < kChunks && ok; ++c) {
       const int st = c % kStages;
       ok = mbar_wait(empty + st, ((c / kStages) & 1) ^ 1, p.e, 0x510);
       if (!ok) break;
       unsigned char *sq = ring + st * kStage;
-      const uint32_t sk = smem_u32(sq + kQTile);
-      if (tid == 0) {
-        mbar_expect_tx(full + st, kQTile);
-        tma_load_2d(sq, &tm_q, full + st, c * 64, t * kH);
+      unsigned char *sk = sq + kQTile;
+      if (lane == 0) mbar_expect_tx(full + st, groups * 512 + (warp == 0 ? kQTile : 0));
+      __syncwarp();
+      if (tid == 0) tma_load_2d(sq, &tm_q, full + st, c * 64, t * kH);
+      if (lane < groups) {
+        const int g = 4 * lane + warp;  // keys 4g .. 4g+3: rows 4g .. 4g+3 of the chunk's tile
+        tma_gather4(sk + g * 512, &tm_kv, full + st, c * 64, rows[4 * g], rows[4 * g + 1], rows[4 * g + 2],
+                    rows[4 * g + 3]);
       }
-      for (int q = tid; q < n * 8; q += kProducers) {
-        const int i = q >> 3, u = q & 7;
-        const long long r = rows[i];
-        const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + c * 128 + u * 16;
-        cp_async16_zfill(sk + sw128_off(i, u), src, r >= 0);
-      }
-      cp_async_arrive_noinc(full + st);
     }
     // value rows: wait until every score MMA has consumed the ring
     if (ok) ok = mbar_wait(s_full, 0, p.e, 0x511);
@@ -187,16 +190,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = vb % kVStages;
       ok = mbar_wait(vempty + st, ((vb / kVStages) & 1) ^ 1, p.e, 0x512);
       if (!ok) break;
-      const uint32_t sv = smem_u32(ring + st * kVBlock);
-      for (int q = tid; q < kVKeys * 64; q += kProducers) {
-        const int i = q >> 6, u = q & 63;
-        const long long r = rows[vb * kVKeys + i];
-        const char *src = kvb + (r >= 0 ? r : 0) * kRowBytes + u * 16;
-        cp_async16_zfill(sv + (u >> 3) * (kVKeys * 128) + sw128_off(i, u & 7), src, r >= 0);
+      // 32 value rows x 8 dim chunks: 64 gathers, 16 per warp; chunk u of the block is
+      // a [32 rows x 128 bytes] tile
+      unsigned char *sv = ring + st * kVBlock;
+      if (lane == 0) mbar_expect_tx(vfull + st, 16 * 512);
+      __syncwarp();
+      if (lane < 16) {
+        const int q = 4 * lane + warp, u = q >> 3, g = q & 7;
+        const int *rg = rows + vb * kVKeys + 4 * g;
+        tma_gather4(sv + u * (kVKeys * 128) + g * 512, &tm_kv, vfull + st, u * 64, rg[0], rg[1], rg[2], rg[3]);
       }
-      cp_async_arrive_noinc(vfull + st);
     }
-    cp_async_wait_all();  // nothing may still land in shared memory after exit
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer
     if (lane == 0) {
@@ -421,6 +425,27 @@ bool make_q_map(CUtensorMap *m, const void *q, unsigned long long rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The latent cache viewed as [rows][576] bf16 for four-row gathers: boxes of 64
+// values x 1 row, 128-byte swizzle (the score and value tiles' layout).
+bool make_kv_gather_map(CUtensorMap *m, const void *kv, unsigned long long rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDk, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Rows of the latent cache under layout L (paged pool or [B][n_max]); 0 when the
+// count does not fit a gather coordinate.
+int kv_rows_of(const Layout &L) {
+  const long long rows = L.page_size ? (long long)L.num_pages * L.page_size : (long long)L.batch * L.n_max;
+  return rows > 0 && rows < 0x7FFFFFFFll ? (int)rows : 0;
+}
+
 size_t part_bytes_per_row(int splits) {
   return (size_t)splits * kH * (kDv * sizeof(__half) + sizeof(float2));
 }
@@ -465,7 +490,9 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
   cudaError_t err = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (err != cudaSuccess) return err;
   Params p;
-  p.kv = static_cast<const __nv_bfloat16 *>(kv);
+  p.kv_rows = kv_rows_of(L);
+  CUtensorMap tkv;
+  if (p.kv_rows == 0 || !make_kv_gather_map(&tkv, kv, (unsigned long long)p.kv_rows)) return cudaErrorInvalidValue;
   p.k = k;
   p.splits = pl.splits;
   p.keys_per_split = pl.keys_per_split;
@@ -483,7 +510,7 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     p.idx = idx + (size_t)r0 * k;
     p.L = L;
     p.L.row0 = L.row0 + r0;
-    err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
+    err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
     if (err != cudaSuccess) return err;
     err = launch_kernel(attn_combine_kernel, dim3(nr, kDv / kCombVals), dim3(128), 0, stream, 0,
                         static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
@@ -554,7 +581,9 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   CUtensorMap tq;
   if (!make_q_map(&tq, q, (unsigned long long)T * kH)) return cudaErrorInvalidValue;
   Params p;
-  p.kv = static_cast<const __nv_bfloat16 *>(kv);
+  p.kv_rows = kv_rows_of(L);
+  CUtensorMap tkv;
+  if (p.kv_rows == 0 || !make_kv_gather_map(&tkv, kv, (unsigned long long)p.kv_rows)) return cudaErrorInvalidValue;
   p.idx = idx;
   p.k = k;
   p.splits = pl.splits;
@@ -566,7 +595,7 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
                                          (size_t)T * pl.splits * kH * kDv * sizeof(__half));
   p.L = L;
   p.e = e;
-  err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, p);
+  err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
   if (err != cudaSuccess) return err;
   return launch_kernel(attn_combine_kernel, dim3(T, kDv / kCombVals), dim3(128), 0, stream, 0,
                        static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
