@@ -14,7 +14,8 @@
 //      and write P = exp(scale (S - max)) as bf16 into shared memory.
 //   3. O[128, 512] = P[128, n] . V[n, 512] with the value rows gathered again
 //      (MN-major B operand, same tile shape); O reuses the TMEM columns S occupied.
-//   4. O (unnormalised), the row max and the row sum go to the workspace; a
+//   4. O, normalised by the split's own sum, is staged as fp16 in the freed score
+//      ring and leaves with bulk stores; the row max and sum go beside it. A
 //      second kernel merges the splits of each row with log-sum-exp weights.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -47,6 +48,8 @@ constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per 
 constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
 constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 4 + 256 + 1024;
 constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
+constexpr int kSlice = kH * 128;               // staged output of 64 values of all heads (fp16)
+static_assert((kDv / 64) * kSlice <= kRing, "the staged output reuses the score ring");
 static_assert(kVStages * kVBlock <= kRing, "value blocks reuse the score ring");
 
 struct Params {
@@ -57,8 +60,9 @@ struct Params {
   int keys_per_split;
   float scale_log2;   // softmax_scale * log2(e)
   float scale;
-  __half *o_part;     // [rows][splits][512 values][128 heads] (head-minor: coalesced stores),
-                      // each split's output normalised by its own softmax sum
+  __half *o_part;     // [rows][splits][8 chunks of 64 values][128 heads][64 values]: each
+                      // split's output normalised by its own softmax sum; the 16-byte
+                      // pieces of a head's 64 values are swizzled (piece ^ (head & 7))
   float2 *ml_part;    // [rows][splits][128]: (max * scale, sum)
   Layout L;
   ErrCtx e;
@@ -78,6 +82,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // the eight softmax/output warps only
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_half(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
@@ -315,9 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       // this warp's 256 output columns, normalised by the split's own sum: a convex
-      // combination of value rows, so fp16 keeps ~1e-3 absolute accuracy. Stores are
-      // head-minor so that each warp writes whole lines.
-      __half *ob = p.o_part + part * (long long)(kDv * kH) + h;
+      // combination of value rows, so fp16 keeps ~1e-3 absolute accuracy. Staged in the
+      // score ring (all its loads have been consumed by now) in the workspace's layout.
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       for (int j = half * 8; j < half * 8 + 8; j += 2) {
         uint32_t v[2][32];
@@ -326,13 +334,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(v[0]);
         tmem_ld_wait(v[1]);
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < 2; ++u) {
+          unsigned char *cb = ring + ((j + u) >> 1) * kSlice + h * 128;  // values 32(j+u) .. +31
 #pragma unroll
-          for (int x = 0; x < 32; ++x) ob[((j + u) * 32 + x) * kH] = __float2half_rn(__uint_as_float(v[u][x]) * inv_l);
+          for (int pc = 0; pc < 4; ++pc) {
+            uint32_t w[4];
+#pragma unroll
+            for (int y = 0; y < 4; ++y)
+              w[y] = pack_half(__uint_as_float(v[u][pc * 8 + 2 * y]) * inv_l,
+                               __uint_as_float(v[u][pc * 8 + 2 * y + 1]) * inv_l);
+            const int piece = ((j + u) & 1) * 4 + pc;
+            *reinterpret_cast<uint4 *>(cb + ((piece ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
       }
+      fence_proxy_async_smem();
       if (half == 0) p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
     } else if (half == 0) {
       p.ml_part[part * kH + h] = make_float2(-INFINITY, 0.f);
+    }
+    softmax_bar();  // the whole output tile is staged
+    if (ok && sw == 0 && lane == 0) {
+      char *dst = reinterpret_cast<char *>(p.o_part + part * (long long)(kDv * kH));
+      for (int c = 0; c < kDv / 64; ++c) bulk_store(dst + c * kSlice, ring + c * kSlice, kSlice);
+      bulk_commit();
+      bulk_wait_read_all();  // the staged tile is read before this CTA ends
     }
   }
   if (error_raised(p.e)) {
@@ -351,48 +377,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the splits of each (row, head) for 8 output values per CTA, one thread per
-// head. With O_c the split's output already divided by its sum l_c:
-// out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c.
-constexpr int kCombVals = 8;
-__global__ void __launch_bounds__(128)
+// Merge the splits of each (row, head). One thread per 16-byte piece of the
+// output (8 values of one head), 256 per CTA, a CTA per quarter of a row's 64-value
+// chunk. With O_c the split's output already divided by its sum l_c and M the
+// largest max of the head over the splits that hold keys:
+// out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c, lse = M + ln(denominator).
+// Each thread forms the weights of its head itself, so that the (max, sum) pairs
+// and the pieces of up to eight splits are all in flight at once.
+constexpr int kCombThreads = 256;
+constexpr int kCombSplits = 8;  // splits loaded together
+__global__ void __launch_bounds__(kCombThreads)
     attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   pdl_prologue();
-  const int t = blockIdx.x, d0 = blockIdx.y * kCombVals, h = threadIdx.x;
+  const int t = blockIdx.x, ch = blockIdx.y >> 2;
+  const int q = (blockIdx.y & 3) * kCombThreads + threadIdx.x, h = q >> 3, piece = q & 7;
   const float2 *ml = ml_part + (long long)t * splits * kH + h;
-  float M = -INFINITY;
-  for (int c = 0; c < splits; ++c) {
-    const float2 v = ml[c * kH];
-    if (v.y > 0.f) M = fmaxf(M, v.x);
-  }
-  float acc[kCombVals];
+  const char *ob = reinterpret_cast<const char *>(o_part + (long long)t * splits * (kDv * kH)) + ch * kSlice +
+                   h * 128 + ((piece ^ (h & 7)) << 4);
+  constexpr long long kSplitBytes = (long long)kDv * kH * 2;
+  float M = -INFINITY, L = 0.f;
+  float acc[8];
 #pragma unroll
-  for (int x = 0; x < kCombVals; ++x) acc[x] = 0.f;
-  float Lsum = 0.f;
-  const __half *ob = o_part + (long long)t * splits * (kDv * kH) + (long long)d0 * kH + h;
-  for (int c0 = 0; c0 < splits; c0 += 4) {
-    float vals[4][kCombVals], wgt[4];
+  for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+  // the running max M changes only between groups of eight splits: the accumulated
+  // sums are rescaled when it does (exactly the single-pass result when splits <= 8)
+  for (int c0 = 0; c0 < splits; c0 += kCombSplits) {
+    float2 v[kCombSplits];
+    uint4 r[kCombSplits];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {  // all loads of four splits in flight together
+    for (int u = 0; u < kCombSplits; ++u) {
       const int c = c0 + u;
-      const float2 v = c < splits ? ml[c * kH] : make_float2(-INFINITY, 0.f);
-      wgt[u] = v.y > 0.f ? __expf(v.x - M) * v.y : 0.f;  // the split's share before normalising
-      Lsum += wgt[u];
-#pragma unroll
-      for (int x = 0; x < kCombVals; ++x)
-        vals[u][x] = wgt[u] != 0.f ? __half2float(__ldcs(ob + (long long)c * (kDv * kH) + x * kH)) : 0.f;
+      v[u] = c < splits ? ml[c * kH] : make_float2(-INFINITY, 0.f);
+      if (c < splits) r[u] = __ldcs(reinterpret_cast<const uint4 *>(ob + c * kSplitBytes));
     }
+    float Mn = M;
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < kCombSplits; ++u)
+      if (v[u].y > 0.f) Mn = fmaxf(Mn, v[u].x);
+    if (Mn != M && M != -INFINITY) {
+      const float f = __expf(M - Mn);
+      L *= f;
 #pragma unroll
-      for (int x = 0; x < kCombVals; ++x) acc[x] = fmaf(wgt[u], vals[u][x], acc[x]);
+      for (int x = 0; x < 8; ++x) acc[x] *= f;
+    }
+    M = Mn;
+#pragma unroll
+    for (int u = 0; u < kCombSplits; ++u) {
+      // a split without keys wrote no output: its weight is 0 and its piece is not read
+      const float w = v[u].y > 0.f ? __expf(v[u].x - M) * v[u].y : 0.f;
+      L += w;
+      if (w == 0.f) continue;
+      const __half2 *hv = reinterpret_cast<const __half2 *>(&r[u]);
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const float2 f = __half22float2(hv[y]);
+        acc[2 * y] = fmaf(w, f.x, acc[2 * y]);
+        acc[2 * y + 1] = fmaf(w, f.y, acc[2 * y + 1]);
+      }
+    }
   }
-  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  *reinterpret_cast<uint4 *>(out + ((long long)t * kH + h) * kDv + d0) =
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  *reinterpret_cast<uint4 *>(out + ((long long)t * kH + h) * kDv + ch * 64 + piece * 8) =
       make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
                  pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
-  if (lse && blockIdx.y == 0) lse[(long long)t * kH + h] = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
+  if (lse && ch == 0 && piece == 0) lse[(long long)t * kH + h] = L > 0.f ? M + logf(L) : -INFINITY;
 }
 
 // ------------------------------------------------------------------ host
@@ -512,7 +561,7 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     p.L.row0 = L.row0 + r0;
     err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
     if (err != cudaSuccess) return err;
-    err = launch_kernel(attn_combine_kernel, dim3(nr, kDv / kCombVals), dim3(128), 0, stream, 0,
+    err = launch_kernel(attn_combine_kernel, dim3(nr, (kDv / 64) * 4), dim3(kCombThreads), 0, stream, 0,
                         static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                         static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
                         lse ? lse + (size_t)r0 * kH : nullptr);
@@ -597,7 +646,7 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   p.e = e;
   err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
   if (err != cudaSuccess) return err;
-  return launch_kernel(attn_combine_kernel, dim3(T, kDv / kCombVals), dim3(128), 0, stream, 0,
+  return launch_kernel(attn_combine_kernel, dim3(T, (kDv / 64) * 4), dim3(kCombThreads), 0, stream, 0,
                        static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                        static_cast<__nv_bfloat16 *>(out), lse);
 }

@@ -1,7 +1,8 @@
 """bf16 tcgen05 sparse MQA attention (128 heads, 576-wide latent rows, 512-wide
 values) against the oracle recomputed on the GPU's own indices: max-abs 2e-2 on
-the output and the log-sum-exp. Decode over contiguous and paged caches, prefill
-with rows shorter than k, index lists with -1 holes, and dsa_forward."""
+the output and the log-sum-exp. Decode over contiguous and paged caches, split
+counts from 1 to 16, prefill with rows shorter than k, index lists with -1 holes,
+and dsa_forward."""
 import numpy as np
 import pytest
 import torch
@@ -52,6 +53,13 @@ def test_attention_decode_contiguous():
 
 def test_attention_decode_paged():
     _stages(W.PAGED_DECODE_128K.replace(batch=3, len_range=None, lens=(4100, 200, 2048)))
+
+
+@pytest.mark.parametrize("k", [600, 1300, 4096])
+def test_attention_split_counts(k):
+    """3, 6 and 16 splits of 256 positions per row (a short last split in the
+    first two), merged by the split-merge kernel."""
+    _stages(W.PAGED_DECODE_128K.replace(batch=3, len_range=None, lens=(k + 3000, 450, k), k=k))
 
 
 def test_attention_prefill_short_rows():
