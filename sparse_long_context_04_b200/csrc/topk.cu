@@ -10,8 +10,10 @@
 // the bin holding the k-th best key. Keys in that bin are the only candidates
 // whose fate is open (about 1% of a long row): every CTA gathers the whole
 // row's candidates and finishes the radix select on them locally (bits 19..10,
-// then 9..0). Selected positions are written in ascending order with warp
-// ballots: keys above the threshold plus the lowest-position keys equal to it.
+// then 9..0). The scan that finds the candidates also lists, per warp and in
+// position order, every key at or above the candidates' bin; the selected ones
+// among them (keys above the threshold plus the lowest-position keys equal to it)
+// are written in ascending order with warp ballots.
 // When the candidates do not fit (very flat score rows) or many keys tie at the
 // threshold, the cluster falls back to full radix passes over all keys. The row
 // is read from memory exactly once.
@@ -44,6 +46,7 @@ constexpr int kAllCap = 2048;   // candidates per row
 constexpr int kLaneCand = kAllCap / kThreads;  // per thread while scanning
 constexpr int kOvfCap = 256;                    // candidates beyond a thread's slots, per CTA
 constexpr int kTieCap = 64;     // keys equal to the threshold resolved on the fast path
+constexpr int kWList = (kBins1 - kBins2) * 2 / kWarps;  // listed keys per warp (in hist1 past bin 1023)
 
 struct Shared {
   unsigned hist1[kBins1];  // this CTA's histogram of bits 31..20, then the cluster totals; later
@@ -60,6 +63,7 @@ struct Shared {
   unsigned wsum2[kWarps];
   unsigned wgt[kWarps];    // per warp segment: keys above the first-pass bin
   unsigned wsel[kWarps];   // per warp segment: selected candidates
+  unsigned wn[kWarps];     // per warp segment: keys at or above the candidates' bin
   uint2 pub;               // (keys above the first-pass bin, candidates) of this CTA, read by the peers
   unsigned cta_cnt[2];     // (greater, equal) counts of this CTA, read by the peers (fallback)
   unsigned sel_before, ntie, novf;
@@ -281,16 +285,24 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
   const int lane = tid & 31, warp = tid >> 5;
   const int seg = ((cnt + kWarps - 1) / kWarps + 127) / 128 * 128;
   const int s0 = min(cnt, warp * seg), s1 = min(cnt, s0 + seg);
+  // hist1 past its first kBins2 bins is free from here on: the per-warp key lists
+  uint16_t *wlist = reinterpret_cast<uint16_t *>(sm.hist1 + kBins2) + warp * kWList;
   {
     const uint32_t above = (b1 << 20) | 0xFFFFFu;  // keys greater than this lie above bin b1
-    unsigned ngt = 0, nc = 0;
+    const uint32_t lowest = b1 << 20;              // keys at or above this: bin b1 or above
+    const unsigned lt = (1u << lane) - 1u;
+    unsigned ngt = 0, nc = 0, wn = 0;
     uint2 *mine = sm.u.allc + tid * kLaneCand;
-    for (int i = s0 + 4 * lane; i < s1; i += 128) {
-      const uint4 q = keys4[i >> 2];
+    for (int i = s0 + 4 * lane; i - 4 * lane < s1; i += 128) {  // the same trip count in every lane
+      const uint4 q = i < s1 ? keys4[i >> 2] : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+      bool ge[4];
+      unsigned m[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const bool ok = i + j < s1;
+        ge[j] = ok && kk[j] >= lowest;
+        m[j] = __ballot_sync(0xFFFFFFFFu, ge[j]);
         ngt += ok && kk[j] > above;
         if (ok && (kk[j] >> 20) == b1) {
           const uint2 c = make_uint2(kk[j], (unsigned)(lo + i + j));
@@ -302,7 +314,20 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
           }
         }
       }
+      const unsigned tot = __popc(m[0]) + __popc(m[1]) + __popc(m[2]) + __popc(m[3]);
+      if (tot == 0u) continue;
+      // listed in position order: lane l's keys 4l .. 4l+3 after those of the lanes below it
+      unsigned at = wn + __popc(m[0] & lt) + __popc(m[1] & lt) + __popc(m[2] & lt) + __popc(m[3] & lt);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (ge[j]) {
+          if (at < (unsigned)kWList) wlist[at] = (uint16_t)(i + j - s0);
+          ++at;
+        }
+      }
+      wn += tot;
     }
+    if (lane == 0) sm.wn[warp] = wn;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ngt += __shfl_xor_sync(0xFFFFFFFFu, ngt, off);
     if (lane == 0) sm.wgt[warp] = ngt;
@@ -441,17 +466,38 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float *__restrict_
     __syncthreads();
     unsigned o = gt_before + sm.sel_before;
     for (int w = 0; w < warp; ++w) o += sm.wgt[w] + sm.wsel[w];
-    // ---- emit this warp's segment in ascending position order, 32 keys per ballot
+    // ---- emit this warp's selected keys in ascending position order, from its list
+    // when every key at or above the candidates' bin fit into it
     const unsigned lt = (1u << lane) - 1u;
-    for (int i = s0 + lane; i - lane < s1; i += 32) {
-      const uint32_t key = i < s1 ? keys[i] : 0u;
-      const bool sel = i < s1 && (key > thr || (key == thr && (uint32_t)(lo + i) <= tcut));
-      const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) {
-        const unsigned at = o + __popc(m & lt);
-        if (at < (unsigned)k) out[at] = (int)(lo + i);
+    const unsigned wn = sm.wn[warp];
+    if (wn <= (unsigned)kWList) {
+      for (unsigned b = 0; b < wn; b += 32) {
+        const unsigned e = b + lane;
+        bool sel = false;
+        int r = 0;
+        if (e < wn) {
+          r = s0 + (int)wlist[e];
+          const uint32_t key = keys[r];
+          sel = key > thr || (key == thr && (uint32_t)(lo + r) <= tcut);
+        }
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+          const unsigned at = o + __popc(m & lt);
+          if (at < (unsigned)k) out[at] = (int)(lo + r);
+        }
+        o += __popc(m);
       }
-      o += __popc(m);
+    } else {
+      for (int i = s0 + lane; i - lane < s1; i += 32) {
+        const uint32_t key = i < s1 ? keys[i] : 0u;
+        const bool sel = i < s1 && (key > thr || (key == thr && (uint32_t)(lo + i) <= tcut));
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+          const unsigned at = o + __popc(m & lt);
+          if (at < (unsigned)k) out[at] = (int)(lo + i);
+        }
+        o += __popc(m);
+      }
     }
     return;
   }

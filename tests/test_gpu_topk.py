@@ -127,3 +127,27 @@ def test_topk_few_ties_at_the_threshold_bit_exact(lens):
         kth = np.sort(row)[::-1][k - 1]
         partial_ties += (row == kth).sum() > k - (row > kth).sum()
     assert partial_ties >= 2  # the case under test: only some of the tied keys are taken
+
+
+@pytest.mark.parametrize("lens", [(131072, 120000, 40000, 9000)])
+def test_topk_sorted_rows_bit_exact(lens):
+    """Rising and falling rows: the best keys crowd into one end of the row, so a
+    few warps hold all the keys at or above the threshold bin (more than their
+    key lists take) while the others hold none."""
+    ensure_lib()
+    k = 2048
+    rng = np.random.default_rng(sum(lens))
+    B = len(lens)
+    n_max = max(lens)
+    ld = (n_max + 3) // 4 * 4
+    host = np.sort(rng.standard_normal((B, ld)), axis=1).astype(np.float32)
+    host[1::2] = host[1::2, ::-1]
+    scores = torch.from_numpy(np.ascontiguousarray(host)).cuda()
+    seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    lay = D.Layout(seq, n_max)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    D.dsa_topk(scores, k, lay, idx)
+    assert D.dsa_get_device_error() == D.DSA_OK
+    got = idx.cpu().numpy()
+    for b, L in enumerate(lens):
+        assert np.array_equal(got[b], O.topk_row(host[b, :L], k)), b
