@@ -378,20 +378,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the splits of each (row, head). One thread per 16-byte piece of the
-// output (8 values of one head), 256 per CTA, a CTA per quarter of a row's 64-value
-// chunk. With O_c the split's output already divided by its sum l_c and M the
+// output (8 values of one head), 128 per CTA, eight CTAs per 64-value chunk of a
+// row. With O_c the split's output already divided by its sum l_c and M the
 // largest max of the head over the splits that hold keys:
 // out = sum_c (e^{m_c - M} l_c) O_c / sum_c e^{m_c - M} l_c, lse = M + ln(denominator).
 // Each thread forms the weights of its head itself, so that the (max, sum) pairs
 // and the pieces of up to eight splits are all in flight at once.
-constexpr int kCombThreads = 256;
-constexpr int kCombSplits = 8;  // splits loaded together
+constexpr int kCombThreads = 128;  // small CTAs: a decode batch's grid fills the GPU in one wave
+constexpr int kCombPer = (kSlice / 16) / kCombThreads;  // CTAs per 64-value chunk of a row
+constexpr int kCombSplits = 8;                          // splits loaded together
 __global__ void __launch_bounds__(kCombThreads)
     attn_combine_kernel(const __half *__restrict__ o_part, const float2 *__restrict__ ml_part, int splits,
                         __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   pdl_prologue();
-  const int t = blockIdx.x, ch = blockIdx.y >> 2;
-  const int q = (blockIdx.y & 3) * kCombThreads + threadIdx.x, h = q >> 3, piece = q & 7;
+  const int t = blockIdx.x, ch = blockIdx.y / kCombPer;
+  const int q = (blockIdx.y % kCombPer) * kCombThreads + threadIdx.x, h = q >> 3, piece = q & 7;
   const float2 *ml = ml_part + (long long)t * splits * kH + h;
   const char *ob = reinterpret_cast<const char *>(o_part + (long long)t * splits * (kDv * kH)) + ch * kSlice +
                    h * 128 + ((piece ^ (h & 7)) << 4);
@@ -561,7 +562,7 @@ cudaError_t launch_attn_bf16(const void *q, const void *kv, int T, float scale, 
     p.L.row0 = L.row0 + r0;
     err = launch_kernel(attn_bf16_kernel, dim3(nr * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
     if (err != cudaSuccess) return err;
-    err = launch_kernel(attn_combine_kernel, dim3(nr, (kDv / 64) * 4), dim3(kCombThreads), 0, stream, 0,
+    err = launch_kernel(attn_combine_kernel, dim3(nr, (kDv / 64) * kCombPer), dim3(kCombThreads), 0, stream, 0,
                         static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                         static_cast<__nv_bfloat16 *>(out) + (size_t)r0 * kH * kDv,
                         lse ? lse + (size_t)r0 * kH : nullptr);
@@ -646,7 +647,7 @@ cudaError_t launch_attn_bf16_noalloc(const void *q, const void *kv, int T, float
   p.e = e;
   err = launch_kernel(attn_bf16_kernel, dim3(T * pl.splits), dim3(kThreads), kSmem, stream, 0, tq, tkv, p);
   if (err != cudaSuccess) return err;
-  return launch_kernel(attn_combine_kernel, dim3(T, (kDv / 64) * 4), dim3(kCombThreads), 0, stream, 0,
+  return launch_kernel(attn_combine_kernel, dim3(T, (kDv / 64) * kCombPer), dim3(kCombThreads), 0, stream, 0,
                        static_cast<const __half *>(p.o_part), static_cast<const float2 *>(p.ml_part), pl.splits,
                        static_cast<__nv_bfloat16 *>(out), lse);
 }
