@@ -92,12 +92,13 @@ def indexer_kl(dc: DeviceCase, idx: torch.Tensor, lse: torch.Tensor, scores: tor
 class Forward:
     """dsa_forward with its buffers allocated once (reusable across steps)."""
 
-    def __init__(self, dc: DeviceCase, keep_idx: bool = True, topk_path: int = D.DSA_TOPK_AUTO):
+    def __init__(self, dc: DeviceCase, keep_idx: bool = True, topk_path: int = D.DSA_TOPK_AUTO,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
         s = dc.inp.spec
         dev = dc.q.device
         self.dc = dc
-        self.out = torch.empty((dc.T, s.H, s.Dv), dtype=dc.q.dtype, device=dev)
-        self.lse = torch.empty((dc.T, s.H), dtype=torch.float32, device=dev)
+        self.out = torch.empty((dc.T, s.H, s.Dv), dtype=dc.q.dtype, device=dev) if out is None else out
+        self.lse = torch.empty((dc.T, s.H), dtype=torch.float32, device=dev) if lse is None else lse
         self.idx = torch.empty((dc.T, s.k), dtype=torch.int32, device=dev) if keep_idx else None
         self.args = D.forward_args(dc.q_idx, dc.q_scale, dc.k_idx, dc.k_scale, dc.w, dc.q, dc.kv, s.k,
                                    s.softmax_scale, dc.layout, self.out, self.lse, self.idx, topk_path)
