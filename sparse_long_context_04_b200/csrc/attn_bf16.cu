@@ -10,13 +10,20 @@
 //   1. S[128 heads, n] = Q_t[128, 576] . K_sel[n, 576]^T  — nine 64-dim chunks,
 //      Q by a tiled TMA load and the selected rows by TMA four-row gathers into
 //      128-byte swizzled tiles; tcgen05 kind::f16, M = 128, N = n, in TMEM.
-//   2. Four warps (one head row per thread) read S from TMEM, take the row max
-//      and write P = exp(scale (S - max)) as bf16 into shared memory.
-//   3. O[128, 512] = P[128, n] . V[n, 512] with the value rows gathered again
-//      (MN-major B operand, same tile shape); O reuses the TMEM columns S occupied.
-//   4. O, normalised by the split's own sum, is staged as fp16 in the freed score
-//      ring and leaves with bulk stores; the row max and sum go beside it. A
-//      second kernel merges the splits of each row with log-sum-exp weights.
+//   2. Eight warps (one head row per thread, two per TMEM lane quadrant) read S
+//      from TMEM, take the row max and write P = exp(scale (S - max)) as bf16 back
+//      into TMEM, where the value MMAs take it as their A operand.
+//   3. O[128, 512] = P[128, n] . V[n, 512], 128 values (two 64-dim chunks, one
+//      MN-major B operand from shared memory) at a time. The key tiles of chunks 6
+//      and 7 are still in the ring when the score MMAs end and serve as the values
+//      384..511 directly; chunks 0+1 are gathered during the score phase into the
+//      shared memory P does not need, chunks 4+5 into the ring's freed query slots,
+//      chunks 2+3 into the space of 6+7 once their MMAs are done.
+//   4. O, normalised by the split's own sum, leaves in two halves, each staged as
+//      fp16 in freed shared memory and written with bulk stores: values 256..511
+//      while the MMAs of values 0..255 run, then values 0..255. The row max and
+//      sum go beside it; a second kernel merges the splits of each row with
+//      log-sum-exp weights.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -37,20 +44,77 @@ constexpr int kStages = 3;
 constexpr int kQTile = kH * 128;               // 16 KiB
 constexpr int kKTile = kMaxKeys * 128;         // 32 KiB
 constexpr int kStage = kQTile + kKTile;        // 48 KiB
-constexpr int kRing = kStages * kStage;        // 144 KiB (later: four 32 KiB value blocks)
-constexpr int kVKeys = 32;                     // value rows per block
-constexpr int kVBlock = kVKeys * kDv * 2;      // 32 KiB
-constexpr int kVStages = 4;
-constexpr int kPBytes = kH * kMaxKeys * 2;     // 64 KiB
+constexpr int kRing = kStages * kStage;        // 144 KiB
+constexpr int kHalfTile = 128 * 128;           // 128 rows of one 64-dim chunk, 16 KiB
+constexpr int kVSlot = 2 * kKTile;             // 64 KiB: value chunks 0 and 1 (the space P would take)
+constexpr uint32_t kPCol = 384;                // TMEM columns of P: 128 (two bf16 per column)
 constexpr int kProducerWarps = 4;              // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per TMEM lane quadrant
 constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
-constexpr int kSmem = 1024 + kRing + kPBytes + kMaxKeys * 4 + 256 + 1024;
+constexpr int kSmem = 1024 + kRing + kVSlot + kMaxKeys * 4 + 256 + 1024;
 constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
-constexpr int kSlice = kH * 128;               // staged output of 64 values of all heads (fp16)
-static_assert((kDv / 64) * kSlice <= kRing, "the staged output reuses the score ring");
-static_assert(kVStages * kVBlock <= kRing, "value blocks reuse the score ring");
+constexpr int kSlice = kH * 128;               // partial output of 64 values of all heads (fp16)
+static_assert(kChunks == 9 && kStages == 3, "the value phase reads chunks 6 and 7 from ring stages 0 and 1");
+
+// Value phase: the pairs of 64-dim chunks in MMA order, where each pair's rows
+// 0..127 and 128..255 lie in shared memory (byte offsets from the ring's start;
+// the second chunk of a pair sits `lbo` bytes after the first, the operand's
+// stride between 64-value groups), and the TMEM column its 128 outputs go to.
+//   pair 0, chunks 6+7: the key tiles of ring stages 0 and 1, left in place;
+//   pair 1, chunks 4+5: the query slots of stages 0 and 1 and stage 2's first
+//                       32 KiB, free once the score MMAs are done;
+//   pair 2, chunks 0+1: the slot after the ring, gathered during the score phase;
+//   pair 3, chunks 2+3: pair 0's space once pair 0's MMAs are done.
+// TMEM: S in columns 0..255 until P is written, P in 384..511; pair 0's outputs in
+// 256..383, pair 1's in 0..127, pair 2's in 128..255, pair 3's in 256..383 once
+// pair 0's have been read out.
+struct VPair {
+  int chunk0;      // first chunk of the pair (values 64 * chunk0 ..)
+  int off0, off1;  // byte offset of the first chunk's rows 0..127 / 128..255
+  int lbo0, lbo1;  // byte distance to the second chunk's rows, per row half
+  uint32_t dcol;   // TMEM column of the pair's first output value
+  __device__ __forceinline__ int off(int h) const { return h ? off1 : off0; }
+  __device__ __forceinline__ int lbo(int h) const { return h ? lbo1 : lbo0; }
+};
+__device__ __forceinline__ VPair vpair(int i) {
+  VPair v;
+  if (i == 0 || i == 3) {  // key tiles of stages 0 and 1: chunk at +16 KiB, rows 128.. at +16 KiB more
+    v.chunk0 = i == 0 ? 6 : 2;
+    v.off0 = kQTile;
+    v.off1 = kQTile + kHalfTile;
+    v.lbo0 = v.lbo1 = kStage;
+    v.dcol = 256;
+  } else if (i == 1) {     // the query slots of stages 0 and 1, and stage 2's first 32 KiB
+    v.chunk0 = 4;
+    v.off0 = 0;
+    v.off1 = 2 * kStage;
+    v.lbo0 = kStage;
+    v.lbo1 = kHalfTile;
+    v.dcol = 0;
+  } else {                 // the slot after the ring: chunk 0 then chunk 1, 32 KiB each
+    v.chunk0 = 0;
+    v.off0 = kRing;
+    v.off1 = kRing + kHalfTile;
+    v.lbo0 = v.lbo1 = kKTile;
+    v.dcol = 128;
+  }
+  return v;
+}
+// TMEM column holding output value d (0..511)
+__device__ __forceinline__ uint32_t out_col(int d) {
+  const int i = d >= 384 ? 0 : d >= 256 ? 1 : d < 128 ? 2 : 3;
+  const VPair v = vpair(i);
+  return v.dcol + (uint32_t)(d - 64 * v.chunk0);
+}
+// Staging of 64-value output chunk c (fp16 [128 heads][64], 16 KiB) before its bulk
+// store: values 256..511 in pair 1's space (free once its MMAs are done), values
+// 0..255 in the slot after the ring (free once every MMA is done).
+__device__ __forceinline__ int stage_off(int c) {
+  if (c < 4) return kRing + c * kSlice;
+  const int i = c - 4;  // query slot of stage 0, of stage 1, then stage 2's first two 16 KiB
+  return i < 2 ? i * kStage : 2 * kStage + (i - 2) * kSlice;
+}
 
 struct Params {
   int kv_rows;        // rows of the latent cache; the gather coordinate of a padding entry
@@ -94,14 +158,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  unsigned char *ring = base;
-  unsigned char *sP = base + kRing;
-  int *rows = reinterpret_cast<int *>(sP + kPBytes);  // gather row of each selected entry
+  unsigned char *ring = base;  // score ring, then value tiles and output staging; the value slot follows it
+  int *rows = reinterpret_cast<int *>(base + kRing + kVSlot);  // gather row of each selected entry
   uint64_t *bars = reinterpret_cast<uint64_t *>(rows + kMaxKeys);
   uint64_t *full = bars, *empty = bars + kStages;
-  uint64_t *vfull = bars + 2 * kStages, *vempty = vfull + kVStages;
-  uint64_t *s_full = vempty + kVStages, *p_full = s_full + 1, *o_full = p_full + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
+  uint64_t *vfull = bars + 2 * kStages;  // value pairs 1..3 gathered
+  uint64_t *vdone = vfull + 4;           // value pair 0 consumed (its space is free)
+  uint64_t *s_full = vdone + 1, *p_full = s_full + 1, *o_hi = p_full + 1, *o_lo = o_hi + 1;
+  uint64_t *hi_read = o_lo + 1;          // the outputs of values 256..511 are out of TMEM
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(hi_read + 1);
   __shared__ int s_nvalid;
   __shared__ uint32_t s_valid[kMaxKeys / 32];  // bit i: selected entry i is a real row
   __shared__ float s_part[2][kH];              // per-half row max, then row sum
@@ -141,21 +206,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x < kH) p.ml_part[part * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
     return;
   }
-  const int n = ((nvalid + 63) / 64) * 64;  // MMA N of the score tile
-  const int nvb = (nvalid + kVKeys - 1) / kVKeys;  // value blocks
+  const int n = ((nvalid + 63) / 64) * 64;  // MMA N of the score tile, K of the value MMAs
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full + s, kProducerWarps);
       mbar_init(empty + s, 1);
     }
-    for (int j = 0; j < kVStages; ++j) {
-      mbar_init(vfull + j, kProducerWarps);
-      mbar_init(vempty + j, 1);
-    }
+    for (int j = 1; j < 4; ++j) mbar_init(vfull + j, kProducerWarps);
+    mbar_init(vdone, 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, kSmWarps);
-    mbar_init(o_full, 1);
+    mbar_init(o_hi, 1);
+    mbar_init(o_lo, 1);
+    mbar_init(hi_read, kSmWarps);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -193,29 +257,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     rows[4 * g + 3]);
       }
     }
-    // value rows: wait until every score MMA has consumed the ring
-    if (ok) ok = mbar_wait(s_full, 0, p.e, 0x511);
-    for (int vb = 0; vb < nvb && ok; ++vb) {
-      const int st = vb % kVStages;
-      ok = mbar_wait(vempty + st, ((vb / kVStages) & 1) ^ 1, p.e, 0x512);
+    // value pairs: 2 now (its slot is free from the start), 1 once every score MMA has
+    // consumed the ring, 3 once pair 0's MMAs have consumed its space
+    for (int k = 0; k < 3 && ok; ++k) {
+      const int i = k == 0 ? 2 : k == 1 ? 1 : 3;
+      if (i == 1) ok = mbar_wait(s_full, 0, p.e, 0x511);
+      if (i == 3) ok = mbar_wait(vdone, 0, p.e, 0x512);
       if (!ok) break;
-      // 32 value rows x 8 dim chunks: 64 gathers, 16 per warp; chunk u of the block is
-      // a [32 rows x 128 bytes] tile
-      unsigned char *sv = ring + st * kVBlock;
-      if (lane == 0) mbar_expect_tx(vfull + st, 16 * 512);
+      const VPair v = vpair(i);
+      // 2 chunks x n/4 row groups; thread q = 4 * lane + warp takes chunk q >> 6, group q & 63
+      const int q = 4 * lane + warp, j = q >> 6, g = q & 63;
+      const bool mine = g < n / 4;
+      const unsigned cnt = __popc(__ballot_sync(0xFFFFFFFFu, mine));
+      if (lane == 0) mbar_expect_tx(vfull + i, cnt * 512);
       __syncwarp();
-      if (lane < 16) {
-        const int q = 4 * lane + warp, u = q >> 3, g = q & 7;
-        const int *rg = rows + vb * kVKeys + 4 * g;
-        tma_gather4(sv + u * (kVKeys * 128) + g * 512, &tm_kv, vfull + st, u * 64, rg[0], rg[1], rg[2], rg[3]);
+      if (mine) {
+        const int h = g >> 5;  // row half
+        unsigned char *dst = ring + v.off(h) + j * v.lbo(h) + (g & 31) * 512;
+        tma_gather4(dst, &tm_kv, vfull + i, (v.chunk0 + j) * 64, rows[4 * g], rows[4 * g + 1], rows[4 * g + 2],
+                    rows[4 * g + 3]);
       }
     }
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, 128, (uint32_t)n);
-      const uint32_t idesc_pv = instr_desc(1, 1, 0, 1, 128, 256);
-      const uint32_t r0 = smem_u32(ring), p0 = smem_u32(sP);
+      const uint32_t r0 = smem_u32(ring);
       bool ok = true;
       for (int c = 0; c < kChunks && ok; ++c) {
         const int st = c % kStages;
@@ -232,25 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(s_full);
       if (ok) ok = mbar_wait(p_full, 0, p.e, 0x521);
       if (ok) tc_fence_after();
-      for (int vb = 0; vb < nvb && ok; ++vb) {
-        const int st = vb % kVStages;
-        ok = mbar_wait(vfull + st, (vb / kVStages) & 1, p.e, 0x522);
-        if (!ok) break;
-        tc_fence_after();
-        // value rows vb*32 .. +31: their P columns sit in 64-key block vb/2, bytes (vb%2)*64 of each row
-        const uint32_t va = r0 + st * kVBlock, pa = p0 + (vb >> 1) * 16384 + (vb & 1) * 64;
-#pragma unroll
-        for (int ks = 0; ks < kVKeys / 16; ++ks) {
-          const uint64_t ad = smem_desc(pa + ks * 32, 16, 1024, SW_128B);
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh)
-            umma_f16(tmem + nh * 256, ad,
-                     smem_desc(va + nh * 4 * (kVKeys * 128) + ks * 2048, kVKeys * 128, 1024, SW_128B), idesc_pv,
-                     (vb | ks) != 0);
+      // O[:, 64 c0 .. 64 c0 + 127] = P . V over n rows in K steps of 16 rows (8 TMEM columns of P each)
+      const uint32_t idesc_pv = instr_desc(1, 1, 0, 1, 128, 128);  // B MN-major, N = 128
+      for (int i = 0; i < 4 && ok; ++i) {
+        if (i > 0) {
+          ok = mbar_wait(vfull + i, 0, p.e, 0x522);
+          if (ok && i == 3) ok = mbar_wait(hi_read, 0, p.e, 0x523);  // pair 3 reuses pair 0's columns
+          if (!ok) break;
+          tc_fence_after();
         }
-        umma_commit(vempty + st);
+        const VPair v = vpair(i);
+        for (int ks = 0; ks < n / 16; ++ks) {
+          const int h = ks >> 3;  // row half
+          const uint64_t bd = smem_desc(r0 + v.off(h) + (ks & 7) * 2048, (uint32_t)v.lbo(h), 1024, SW_128B);
+          umma_f16_ts(tmem + v.dcol, tmem + kPCol + ks * 8, bd, idesc_pv, ks != 0);
+        }
+        if (i == 0) umma_commit(vdone);
+        if (i == 1) umma_commit(o_hi);  // values 256..511 complete
       }
-      umma_commit(o_full);
+      umma_commit(o_lo);  // every MMA of this CTA complete
     }
     __syncwarp();
   } else {
@@ -304,15 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat162 bw = *reinterpret_cast<const __nv_bfloat162 *>(&w);
           l += __low2float(bw) + __high2float(bw);
         }
-        // keys j*32 .. j*32+31 sit in 64-key block j/2, 16-byte chunks (j%2)*4 .. +3
-        unsigned char *pb = sP + (j >> 1) * 16384;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const uint32_t off = sw128_off((uint32_t)h, (uint32_t)((j & 1) * 4 + c4));
-          *reinterpret_cast<uint4 *>(pb + off) = make_uint4(pk[c4 * 4], pk[c4 * 4 + 1], pk[c4 * 4 + 2], pk[c4 * 4 + 3]);
-        }
+        // keys j*32 .. j*32+31: 16 TMEM columns of P, two keys per column
+        tmem_st16(trow + kPCol + j * 16, pk);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
@@ -320,46 +382,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_part[half][h] = l;
     softmax_bar();
     l = s_part[0][h] + s_part[1][h];
-    if (ok) ok = mbar_wait(o_full, 0, p.e, 0x531);
-    if (ok) {
-      tc_fence_after();
-      // this warp's 256 output columns, normalised by the split's own sum: a convex
-      // combination of value rows, so fp16 keeps ~1e-3 absolute accuracy. Staged in the
-      // score ring (all its loads have been consumed by now) in the workspace's layout.
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      for (int j = half * 8; j < half * 8 + 8; j += 2) {
-        uint32_t v[2][32];
-        tmem_ld32(trow + j * 32, v[0]);
-        tmem_ld32(trow + (j + 1) * 32, v[1]);
-        tmem_ld_wait(v[0]);
-        tmem_ld_wait(v[1]);
+    // this warp's 256 output values in two halves, normalised by the split's own sum
+    // (a convex combination of value rows, so fp16 keeps ~1e-3 absolute accuracy):
+    // staged in the workspace's layout (64-value chunks of [128 heads][64], the
+    // 16-byte pieces of a head swizzled by the head's low three bits), then bulk stores
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    char *ob = reinterpret_cast<char *>(p.o_part + part * (long long)(kDv * kH));
+    for (int hv = 1; hv >= 0; --hv) {  // values 256..511 first, then 0..255
+      if (ok) ok = mbar_wait(hv ? o_hi : o_lo, 0, p.e, 0x531);
+      if (ok) {
+        tc_fence_after();
+        const int d0 = hv * 256 + half * 128;  // this warp's 128 values
+        for (int d = d0; d < d0 + 128; d += 64) {
+          uint32_t v[2][32];
+          tmem_ld32(trow + out_col(d), v[0]);
+          tmem_ld32(trow + out_col(d + 32), v[1]);
+          tmem_ld_wait(v[0]);
+          tmem_ld_wait(v[1]);
+          unsigned char *cb = ring + stage_off(d >> 6) + h * 128;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          unsigned char *cb = ring + ((j + u) >> 1) * kSlice + h * 128;  // values 32(j+u) .. +31
+          for (int u = 0; u < 2; ++u) {
 #pragma unroll
-          for (int pc = 0; pc < 4; ++pc) {
-            uint32_t w[4];
+            for (int pc = 0; pc < 4; ++pc) {
+              uint32_t w[4];
 #pragma unroll
-            for (int y = 0; y < 4; ++y)
-              w[y] = pack_half(__uint_as_float(v[u][pc * 8 + 2 * y]) * inv_l,
-                               __uint_as_float(v[u][pc * 8 + 2 * y + 1]) * inv_l);
-            const int piece = ((j + u) & 1) * 4 + pc;
-            *reinterpret_cast<uint4 *>(cb + ((piece ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int y = 0; y < 4; ++y)
+                w[y] = pack_half(__uint_as_float(v[u][pc * 8 + 2 * y]) * inv_l,
+                                 __uint_as_float(v[u][pc * 8 + 2 * y + 1]) * inv_l);
+              const int piece = u * 4 + pc;
+              *reinterpret_cast<uint4 *>(cb + ((piece ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      if (half == 0) p.ml_part[part * kH + h] = make_float2(m * p.scale, l);
-    } else if (half == 0) {
-      p.ml_part[part * kH + h] = make_float2(-INFINITY, 0.f);
+      if (hv) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hi_read);  // pair 3 may overwrite these TMEM columns
+      }
+      softmax_bar();  // the half is staged
+      if (ok && sw == 0 && lane == 0) {
+        for (int c = hv * 4; c < hv * 4 + 4; ++c) bulk_store(ob + c * kSlice, ring + stage_off(c), kSlice);
+        bulk_commit();
+      }
     }
-    softmax_bar();  // the whole output tile is staged
-    if (ok && sw == 0 && lane == 0) {
-      char *dst = reinterpret_cast<char *>(p.o_part + part * (long long)(kDv * kH));
-      for (int c = 0; c < kDv / 64; ++c) bulk_store(dst + c * kSlice, ring + c * kSlice, kSlice);
-      bulk_commit();
-      bulk_wait_read_all();  // the staged tile is read before this CTA ends
-    }
+    if (sw == 0 && lane == 0) bulk_wait_read_all();  // the staged tiles are read before this CTA ends
+    if (half == 0) p.ml_part[part * kH + h] = ok ? make_float2(m * p.scale, l) : make_float2(-INFINITY, 0.f);
   }
   if (error_raised(p.e)) {
     // a wait gave up somewhere: copies and MMAs issued before that may still be in flight
@@ -370,8 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) {
-    // all MMAs have completed once o_full fired; if a wait gave up, wait here (bounded)
-    if (lane == 0) mbar_wait(o_full, 0, p.e, 0x540);
+    // all MMAs have completed once o_lo fired; if a wait gave up, wait here (bounded)
+    if (lane == 0) mbar_wait(o_lo, 0, p.e, 0x540);
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
