@@ -19,11 +19,11 @@
 //      384..511 directly; chunks 0+1 are gathered during the score phase into the
 //      shared memory P does not need, chunks 4+5 into the ring's freed query slots,
 //      chunks 2+3 into the space of 6+7 once their MMAs are done.
-//   4. O, normalised by the split's own sum, leaves in two halves, each staged as
-//      fp16 in freed shared memory and written with bulk stores: values 256..511
-//      while the MMAs of values 0..255 run, then values 0..255. The row max and
-//      sum go beside it; a second kernel merges the splits of each row with
-//      log-sum-exp weights.
+//   4. O, normalised by the split's own sum, leaves in three parts as each is
+//      complete, each staged as fp16 in freed shared memory and written with bulk
+//      stores: values 256..511 and then 0..127 while later MMAs run, 128..255 last.
+//      The row max and sum go beside it; a second kernel merges the splits of each
+//      row with log-sum-exp weights.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -164,7 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *full = bars, *empty = bars + kStages;
   uint64_t *vfull = bars + 2 * kStages;  // value pairs 1..3 gathered
   uint64_t *vdone = vfull + 4;           // value pair 0 consumed (its space is free)
-  uint64_t *s_full = vdone + 1, *p_full = s_full + 1, *o_hi = p_full + 1, *o_lo = o_hi + 1;
+  uint64_t *s_full = vdone + 1, *p_full = s_full + 1;
+  uint64_t *o_done = p_full + 1;         // outputs complete: values 256..511, 0..127, 128..255
+  uint64_t *o_lo = o_done + 2;           // (the last one: every MMA of this CTA complete)
   uint64_t *hi_read = o_lo + 1;          // the outputs of values 256..511 are out of TMEM
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(hi_read + 1);
   __shared__ int s_nvalid;
@@ -217,8 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(vdone, 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, kSmWarps);
-    mbar_init(o_hi, 1);
-    mbar_init(o_lo, 1);
+    for (int j = 0; j < 3; ++j) mbar_init(o_done + j, 1);
     mbar_init(hi_read, kSmWarps);
     fence_mbar_init();
   }
@@ -315,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_f16_ts(tmem + v.dcol, tmem + kPCol + ks * 8, bd, idesc_pv, ks != 0);
         }
         if (i == 0) umma_commit(vdone);
-        if (i == 1) umma_commit(o_hi);  // values 256..511 complete
+        if (i == 1) umma_commit(o_done);      // values 256..511 complete
+        if (i == 2) umma_commit(o_done + 1);  // values 0..127 complete
       }
       umma_commit(o_lo);  // every MMA of this CTA complete
     }
@@ -382,18 +384,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_part[half][h] = l;
     softmax_bar();
     l = s_part[0][h] + s_part[1][h];
-    // this warp's 256 output values in two halves, normalised by the split's own sum
+    // this warp's 256 output values in three parts, normalised by the split's own sum
     // (a convex combination of value rows, so fp16 keeps ~1e-3 absolute accuracy):
     // staged in the workspace's layout (64-value chunks of [128 heads][64], the
     // 16-byte pieces of a head swizzled by the head's low three bits), then bulk stores
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     char *ob = reinterpret_cast<char *>(p.o_part + part * (long long)(kDv * kH));
-    for (int hv = 1; hv >= 0; --hv) {  // values 256..511 first, then 0..255
-      if (ok) ok = mbar_wait(hv ? o_hi : o_lo, 0, p.e, 0x531);
+    for (int pt = 0; pt < 3; ++pt) {  // values 256..511, then 0..127, then 128..255
+      const int lo = pt == 0 ? 256 : pt == 1 ? 0 : 128, width = pt == 0 ? 256 : 128;
+      if (ok) ok = mbar_wait(pt == 2 ? o_lo : o_done + pt, 0, p.e, 0x531);
       if (ok) {
         tc_fence_after();
-        const int d0 = hv * 256 + half * 128;  // this warp's 128 values
-        for (int d = d0; d < d0 + 128; d += 64) {
+        const int d0 = lo + half * (width / 2);  // this warp's values
+        for (int d = d0; d < d0 + width / 2; d += 64) {
           uint32_t v[2][32];
           tmem_ld32(trow + out_col(d), v[0]);
           tmem_ld32(trow + out_col(d + 32), v[1]);
@@ -416,14 +419,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
       }
-      if (hv) {
+      if (pt == 0) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(hi_read);  // pair 3 may overwrite these TMEM columns
       }
-      softmax_bar();  // the half is staged
+      softmax_bar();  // the part is staged
       if (ok && sw == 0 && lane == 0) {
-        for (int c = hv * 4; c < hv * 4 + 4; ++c) bulk_store(ob + c * kSlice, ring + stage_off(c), kSlice);
+        for (int c = lo / 64; c < (lo + width) / 64; ++c) bulk_store(ob + c * kSlice, ring + stage_off(c), kSlice);
         bulk_commit();
       }
     }
