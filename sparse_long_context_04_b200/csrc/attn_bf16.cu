@@ -52,6 +52,7 @@ constexpr int kProducerWarps = 4;              // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per TMEM lane quadrant
 constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
+static_assert(kThreads >= kMaxKeys, "one selection entry per thread");
 constexpr int kSmem = 1024 + kRing + kVSlot + kMaxKeys * 4 + 256 + 1024;
 constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
 constexpr int kSlice = kH * 128;               // partial output of 64 values of all heads (fp16)
@@ -181,18 +182,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = min(p.keys_per_split, p.k - k0);
   const long long part = (long long)t * p.splits + split;
 
-  // ---- selected rows of this split (-1 entries are padding, anywhere in the list)
-  if (threadIdx.x == 0) s_nvalid = 0;
+  // ---- barriers and TMEM (they do not depend on the selection, so they overlap
+  // its loads), then the selected rows of this split (-1 entries are padding,
+  // anywhere in the list)
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, kProducerWarps);
+      mbar_init(empty + s, 1);
+    }
+    for (int j = 1; j < 4; ++j) mbar_init(vfull + j, kProducerWarps);
+    mbar_init(vdone, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, kSmWarps);
+    for (int j = 0; j < 3; ++j) mbar_init(o_done + j, 1);
+    mbar_init(hi_read, kSmWarps);
+    fence_mbar_init();
+    s_nvalid = 0;
+  }
   if (threadIdx.x < kMaxKeys / 32) s_valid[threadIdx.x] = 0;
-  __syncthreads();
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
   const RowPos rp = row_position(p.L, t);
-  for (int i = threadIdx.x; i < kMaxKeys; i += kThreads) {
+  const int i = threadIdx.x;  // entry i of the split's selection (kThreads >= kMaxKeys)
+  const int sel = i < nk && i < kMaxKeys ? __ldg(p.idx + (long long)t * p.k + k0 + i) : -1;
+  tc_fence_before();
+  __syncthreads();  // s_nvalid, s_valid and the barriers are initialised
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (i < kMaxKeys) {
     long long r = -1;
     if (i < nk) {
-      const int s = __ldg(p.idx + (long long)t * p.k + k0 + i);
-      if (s >= 0 && s <= rp.pos && rp.len <= cache_capacity(p.L)) {
-        r = key_row(p.L, rp.b, s, p.e, 0x500);
-      } else if (s != -1) {
+      if (sel >= 0 && sel <= rp.pos && rp.len <= cache_capacity(p.L)) {
+        r = key_row(p.L, rp.b, sel, p.e, 0x500);
+      } else if (sel != -1) {
         raise_error(p.e, DEV_BOUNDS, 0x501);
       }
     }
@@ -206,31 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nvalid = s_nvalid;  // entries at or after nvalid are all padding
   if (nvalid == 0) {
     if (threadIdx.x < kH) p.ml_part[part * kH + threadIdx.x] = make_float2(-INFINITY, 0.f);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
     return;
   }
   const int n = ((nvalid + 63) / 64) * 64;  // MMA N of the score tile, K of the value MMAs
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full + s, kProducerWarps);
-      mbar_init(empty + s, 1);
-    }
-    for (int j = 1; j < 4; ++j) mbar_init(vfull + j, kProducerWarps);
-    mbar_init(vdone, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, kSmWarps);
-    for (int j = 0; j < 3; ++j) mbar_init(o_done + j, 1);
-    mbar_init(hi_read, kSmWarps);
-    fence_mbar_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp < kProducerWarps) {
     // ================= producers: Q chunks by a tiled TMA load, selected rows by
@@ -344,9 +347,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < 2; ++u) {
           if (j + u >= j1) break;
           const uint32_t vm = s_valid[j + u];
+          if (vm == 0xFFFFFFFFu) {  // every entry of the chunk is a real row: a plain tree
+            float t8[8];
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if ((vm >> x) & 1u) m = fmaxf(m, __uint_as_float(v[u][x]));
+            for (int y = 0; y < 8; ++y)
+              t8[y] = fmaxf(fmaxf(__uint_as_float(v[u][4 * y]), __uint_as_float(v[u][4 * y + 1])),
+                            fmaxf(__uint_as_float(v[u][4 * y + 2]), __uint_as_float(v[u][4 * y + 3])));
+            m = fmaxf(m, fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                               fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7]))));
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if ((vm >> x) & 1u) m = fmaxf(m, __uint_as_float(v[u][x]));
+          }
         }
       }
     }
