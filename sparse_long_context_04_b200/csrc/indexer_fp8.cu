@@ -344,6 +344,34 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.L.batch;
 
+  // ---- barriers and TMEM (independent of the work range, so set up while its loads run)
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(a_full + st, 1);
+      mbar_init(a_empty + st, 1 + C::kWarpsPerItem);  // the MMA commit and the tile's epilogue warps
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(b_full + j, 1);
+      mbar_init(b_empty + j, C::kMmaWarps + C::kEpiWarps);  // every MMA and epilogue warp
+    }
+    for (int j = 0; j < C::kAccBufs; ++j) {
+      mbar_init(acc_full + j, 1);
+      mbar_init(acc_empty + j, C::kWarpsPerItem);
+    }
+    for (int j = 0; j < C::kMmaWarps; ++j) mbar_init(done_bar + j, 1);
+    s_b_turn = 0;
+    s_bound = 0ull;
+    s_top = 0ull;
+    s_cur_row = -1;
+    s_tiles = 0;
+    s_epi_done = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::kMmaWarp0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   // ---- work range: per-sequence item counts (closed form), block prefix sum
   {
     long long *pre = reinterpret_cast<long long *>(sA);  // aliases stage memory before any load
@@ -408,37 +436,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     __syncthreads();
   }
   const long long n_items = s_range[1];
-
-  // ---- barriers and TMEM
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < C::kStages; ++st) {
-      mbar_init(a_full + st, 1);
-      mbar_init(a_empty + st, 1 + C::kWarpsPerItem);  // the MMA commit and the tile's epilogue warps
-    }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(b_full + j, 1);
-      mbar_init(b_empty + j, C::kMmaWarps + C::kEpiWarps);  // every MMA and epilogue warp
-    }
-    for (int j = 0; j < C::kAccBufs; ++j) {
-      mbar_init(acc_full + j, 1);
-      mbar_init(acc_empty + j, C::kWarpsPerItem);
-    }
-    for (int j = 0; j < C::kMmaWarps; ++j) mbar_init(done_bar + j, 1);
-    s_b_turn = 0;
-    s_bound = 0ull;
-    s_top = 0ull;
-    s_cur_row = -1;
-    s_tiles = 0;
-    s_epi_done = 0;
-    fence_mbar_init();
-  }
-  if (warp == C::kMmaWarp0) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  tc_fence_after();  // the work range's block barriers also ordered the TMEM allocation
   const uint32_t tmem = *tmem_slot;
 
   if (n_items > 0) {
