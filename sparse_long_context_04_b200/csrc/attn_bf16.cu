@@ -110,7 +110,8 @@ __device__ __forceinline__ uint32_t out_col(int d) {
 }
 // Staging of 64-value output chunk c (fp16 [128 heads][64], 16 KiB) before its bulk
 // store: values 256..511 in pair 1's space (free once its MMAs are done), values
-// 0..255 in the slot after the ring (free once every MMA is done).
+// 0..255 in the slot after the ring, pair 2's space (free once pair 2's MMAs are
+// done; values 0..127 are staged then, 128..255 after the last MMA).
 __device__ __forceinline__ int stage_off(int c) {
   if (c < 4) return kRing + c * kSlice;
   const int i = c - 4;  // query slot of stage 0, of stage 1, then stage 2's first two 16 KiB
