@@ -312,7 +312,9 @@ __device__ int row_bound(const Params &p, int t, int cur, int top) {
 }
 
 // ------------------------------------------------------------------ kernel
-template <int G>
+// F: the fused top-k's producer (decode only) instead of score rows; a template
+// argument so that the score-row kernel carries none of its branches or state.
+template <int G, bool F>
 __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const Params p) {
@@ -591,7 +593,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     } else if (G == 1 && warp == C::kBoundWarp) {
       // ================= bound warp (fused top-k): about once a microsecond, a fresh
       // lower bound of the current row's threshold bin from the global histograms
-      if (p.fuse) {
+      if (F) {
         const unsigned long long t0 = globaltimer();
         int seen = -1;  // tiles finished at the last refresh: refresh only after new ones
         while (*reinterpret_cast<volatile int *>(&s_epi_done) < C::kEpiWarps) {
@@ -719,7 +721,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
               const int t = cur.row0() + gi;
               const float v = acc * qs[tt] * sk;
               const bool valid = gi < nrows && key_ok && s <= pos;
-              if (G == 1 && p.fuse) {
+              if (G == 1 && F) {
                 // the candidates at or above the current bound and their histogram
                 // (fire-and-forget atomics), instead of the scores
                 const uint32_t bin = order_key(v) >> 20;
@@ -761,7 +763,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           if (lane == 0) mbar_arrive(b_empty + slot);
         }
       }
-      if (G == 1 && p.fuse) flush_pending();
+      if (G == 1 && F) flush_pending();
       __syncwarp();
       if (lane == 0) atomicAdd(&s_epi_done, 1);  // the bound warp stops once all have finished
     }
@@ -807,7 +809,7 @@ bool make_map(CUtensorMap *m, const void *ptr, unsigned long long rows, unsigned
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G>
+template <int G, bool F>
 cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int num_sms, cudaStream_t stream) {
   using C = Cfg<G>;
   CUtensorMap tq, tk;
@@ -816,9 +818,10 @@ cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int n
   if (!make_map(&tq, q, (unsigned long long)p.T * kHI, C::N)) return cudaErrorInvalidValue;
   if (!make_map(&tk, kI, krows, 64)) return cudaErrorInvalidValue;
   cudaError_t err =
-      cudaFuncSetAttribute(indexer_fp8_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      cudaFuncSetAttribute(indexer_fp8_kernel<G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (err != cudaSuccess) return err;
-  return launch_kernel(indexer_fp8_kernel<G>, dim3(num_sms), dim3(C::kThreads), C::kSmem, stream, 0, tq, tk, p);
+  return launch_kernel(indexer_fp8_kernel<G, F>, dim3(num_sms), dim3(C::kThreads), C::kSmem, stream, 0, tq, tk,
+                       p);
 }
 
 }  // namespace
@@ -848,8 +851,8 @@ cudaError_t launch_indexer_fp8(const uint8_t *q, const float *q_scale, const uin
   p.cand_score = nullptr;
   p.cand_pos = nullptr;
   p.cand_cap = 0;
-  if (L.cu_q == nullptr) return launch_g<1>(q, kI, p, num_sms, stream);
-  return launch_g<4>(q, kI, p, num_sms, stream);
+  if (L.cu_q == nullptr) return launch_g<1, false>(q, kI, p, num_sms, stream);
+  return launch_g<4, false>(q, kI, p, num_sms, stream);
 }
 
 namespace {
@@ -894,7 +897,7 @@ cudaError_t launch_indexer_fp8_fused(const uint8_t *q, const float *q_scale, con
   p.cand_score = cand_score;
   p.cand_pos = cand_pos;
   p.cand_cap = cand_cap;
-  return launch_g<1>(q, kI, p, num_sms, stream);
+  return launch_g<1, true>(q, kI, p, num_sms, stream);
 }
 
 }  // namespace dsa
