@@ -232,8 +232,8 @@ def main():
     cand_s = torch.empty((T, dc.ld), dtype=torch.float32, device=dev)
     cand_p = torch.empty((T, dc.ld), dtype=torch.int32, device=dev)
     cand_n = torch.empty((T,), dtype=torch.int32, device=dev)
-    # indexer, top-k, then attention: a kernel and a split-merge kernel per chunk of 296 rows
-    launches_per_step = 2 + 2 * ((T + 295) // 296)
+    # indexer, top-k, then attention: a kernel and a split-merge kernel per chunk of 74 rows
+    launches_per_step = 2 + 2 * ((T + 73) // 74)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):

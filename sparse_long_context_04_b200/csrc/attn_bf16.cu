@@ -54,7 +54,8 @@ constexpr int kSmWarp0 = 5, kSmWarps = 8;      // softmax/output warps: two per 
 constexpr int kThreads = 32 * (4 + 1 + kSmWarps);
 static_assert(kThreads >= kMaxKeys, "one selection entry per thread");
 constexpr int kSmem = 1024 + kRing + kVSlot + kMaxKeys * 4 + 256 + 1024;
-constexpr int kRowsPerLaunch = 296;            // bounds the partial-result workspace
+constexpr int kRowsPerLaunch = 74;             // rows per launch: 74 x 8 splits = four waves of 148 CTAs, and
+                                               // the launch's fp16 partials (74 MB) stay in L2 for the merge
 constexpr int kSlice = kH * 128;               // partial output of 64 values of all heads (fp16)
 static_assert(kChunks == 9 && kStages == 3, "the value phase reads chunks 6 and 7 from ring stages 0 and 1");
 
