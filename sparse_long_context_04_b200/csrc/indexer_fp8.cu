@@ -312,9 +312,10 @@ __device__ int row_bound(const Params &p, int t, int cur, int top) {
 }
 
 // ------------------------------------------------------------------ kernel
-// F: the fused top-k's producer (decode only) instead of score rows; a template
-// argument so that the score-row kernel carries none of its branches or state.
-template <int G, bool F>
+// F: the fused top-k's producer (decode only) instead of score rows; PG: the key
+// cache is paged (its scales always come by bulk copy). Template arguments so that
+// each kernel carries only its own branches and state.
+template <int G, bool F, bool PG>
 __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
     indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const Params p) {
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
                 int y0 = -1, y1 = -1;
                 const unsigned char *sc0 = nullptr, *sc1 = nullptr;
                 uint32_t sb0 = 0, sb1 = 0;
-                if (p.L.page_size == 0) {
+                if (!PG) {
                   y0 = (int)((long long)b * p.L.n_max + s0);
                   y1 = y0 + 64;
                   if (p.scales_bulk) {
@@ -672,7 +673,7 @@ __global__ void __launch_bounds__(Cfg<G>::kThreads, 1)
           const int b = cur.b;
           const bool key_ok = s < cur.s.len;
           float sk = 0.f;
-          if (p.scales_bulk) {
+          if (PG || p.scales_bulk) {
             sk = sScale[st * kTileKeys + r];
           } else if (key_ok) {
             if (p.L.page_size == 0) {
@@ -809,8 +810,8 @@ bool make_map(CUtensorMap *m, const void *ptr, unsigned long long rows, unsigned
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G, bool F>
-cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int num_sms, cudaStream_t stream) {
+template <int G, bool F, bool PG>
+cudaError_t launch_gp(const uint8_t *q, const uint8_t *kI, const Params &p, int num_sms, cudaStream_t stream) {
   using C = Cfg<G>;
   CUtensorMap tq, tk;
   const unsigned long long krows =
@@ -818,10 +819,15 @@ cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int n
   if (!make_map(&tq, q, (unsigned long long)p.T * kHI, C::N)) return cudaErrorInvalidValue;
   if (!make_map(&tk, kI, krows, 64)) return cudaErrorInvalidValue;
   cudaError_t err =
-      cudaFuncSetAttribute(indexer_fp8_kernel<G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      cudaFuncSetAttribute(indexer_fp8_kernel<G, F, PG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (err != cudaSuccess) return err;
-  return launch_kernel(indexer_fp8_kernel<G, F>, dim3(num_sms), dim3(C::kThreads), C::kSmem, stream, 0, tq, tk,
-                       p);
+  return launch_kernel(indexer_fp8_kernel<G, F, PG>, dim3(num_sms), dim3(C::kThreads), C::kSmem, stream, 0, tq,
+                       tk, p);
+}
+template <int G, bool F>
+cudaError_t launch_g(const uint8_t *q, const uint8_t *kI, const Params &p, int num_sms, cudaStream_t stream) {
+  return p.L.page_size ? launch_gp<G, F, true>(q, kI, p, num_sms, stream)
+                       : launch_gp<G, F, false>(q, kI, p, num_sms, stream);
 }
 
 }  // namespace
